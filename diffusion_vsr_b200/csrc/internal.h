@@ -1,0 +1,66 @@
+// Kernel argument blocks and launchers shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace lcsa {
+
+constexpr int kBlockTokens = 128;
+constexpr int kHeadDim = 128;
+constexpr int kMaxAppendLayers = 16;
+constexpr int kMaxCandidates = 4096;
+constexpr uint64_t kWatchdogNs = 4000000000ull;  // 4 s per bounded wait
+
+// Block-sparse attention (tcgen05 kernel).
+struct AttnArgs {
+    int32_t heads, grid_h, grid_w, nblk, q_layers, tq;  // tq = 2 * q_layers frames
+    int32_t tok_h, tok_w;
+    int32_t n_key_blocks;  // count * nblk
+    int32_t capacity, oldest;
+    int32_t topk;
+    int32_t n_units;       // heads * q_layers * nblk
+    float scale_log2;      // softmax scale * log2(e)
+    const int32_t *kept_idx;
+    const int32_t *kept_cnt;
+    float *lse;            // may be null
+    int32_t *status;       // may be null
+    uint64_t timeout_ns;
+    int32_t flags;
+};
+
+cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                             const CUtensorMap &tm_o, const AttnArgs &a, cudaStream_t stream);
+
+// Draft mask: q block means, scores over allowed candidates, top-k.
+struct DraftArgs {
+    const uint16_t *q;     // bf16 token layout
+    const float *kmean;    // [cap][H][nblk][128]
+    int32_t heads, grid_h, grid_w, nblk, q_layers, tq, tok_h, tok_w;
+    int32_t capacity, oldest, count;
+    int32_t local_range, local_mode, topk;
+    float scale;
+    int32_t *kept_idx;
+    int32_t *kept_cnt;
+    float *scores;         // may be null
+    float *qmean;          // may be null
+    int32_t *status;
+};
+
+cudaError_t launch_draft(const DraftArgs &a, cudaStream_t stream);
+
+// Cache append: token layout -> block layout ring slots + k block means.
+struct AppendArgs {
+    const uint16_t *k_tok;
+    const uint16_t *v_tok;
+    uint16_t *k_cache;
+    uint16_t *v_cache;
+    float *kmean;
+    int32_t heads, grid_h, grid_w, nblk, tok_h, tok_w, n_layers;
+    int32_t slots[kMaxAppendLayers];
+};
+
+cudaError_t launch_cache_append(const AppendArgs &a, cudaStream_t stream);
+
+}  // namespace lcsa

@@ -1,0 +1,262 @@
+// C ABI of the LCSA library: argument validation, TMA tensor maps, launches.
+// Declarations and the meaning of every argument: include/lcsa.h.
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "../../include/lcsa.h"
+
+namespace {
+
+using lcsa::kBlockTokens;
+using lcsa::kHeadDim;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Only compute capability 10.0 (B200, sm_100a code) is supported.
+int check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LCSA_ERR_CUDA;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return LCSA_ERR_CUDA;
+    if (major != 10 || minor != 0) return LCSA_ERR_UNSUPPORTED_DEVICE;
+    return LCSA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cache(const lcsa_kv_cache *c) {
+    if (!c || !c->k || !c->v || !c->kmean) return LCSA_ERR_INVALID_ARG;
+    if (!aligned16(c->k) || !aligned16(c->v) || !aligned16(c->kmean)) return LCSA_ERR_INVALID_ARG;
+    if (c->heads < 1 || c->grid_h < 1 || c->grid_w < 1 || c->capacity < 1) return LCSA_ERR_INVALID_ARG;
+    if (c->count < 0 || c->count > c->capacity || c->oldest < 0 || c->oldest >= c->capacity)
+        return LCSA_ERR_INVALID_ARG;
+    // every token row index of the ring must fit a signed 32-bit TMA coordinate
+    const int64_t rows = static_cast<int64_t>(c->capacity) * c->heads * c->grid_h * c->grid_w * kBlockTokens;
+    if (rows >= (int64_t(1) << 31)) return LCSA_ERR_INVALID_ARG;
+    return LCSA_OK;
+}
+
+int check_params(const lcsa_params *p, const lcsa_kv_cache *c) {
+    if (!p) return LCSA_ERR_INVALID_ARG;
+    if (p->head_dim != kHeadDim) return LCSA_ERR_INVALID_ARG;
+    if (p->heads < 1 || p->grid_h < 1 || p->grid_w < 1 || p->q_layers < 1 || p->topk < 1) return LCSA_ERR_INVALID_ARG;
+    if (p->local_mode != 0 && p->local_mode != 1) return LCSA_ERR_INVALID_ARG;
+    if (p->local_range > 0 && (p->local_range % 2) == 0) return LCSA_ERR_INVALID_ARG;
+    if (!(p->scale >= 0.f) || std::isinf(p->scale)) return LCSA_ERR_INVALID_ARG;
+    if (p->heads != c->heads || p->grid_h != c->grid_h || p->grid_w != c->grid_w) return LCSA_ERR_INVALID_ARG;
+    if (c->count < p->q_layers) return LCSA_ERR_INVALID_ARG;
+    // frames * tokens must be addressable by 32-bit TMA coordinates
+    const int64_t frames = static_cast<int64_t>(p->heads) * 2 * p->q_layers;
+    if (frames >= (int64_t(1) << 31) || 8LL * p->grid_h >= (1 << 30) || 8LL * p->grid_w >= (1 << 30))
+        return LCSA_ERR_INVALID_ARG;
+    return LCSA_OK;
+}
+
+float eff_scale(const lcsa_params *p) {
+    return p->scale > 0.f ? p->scale : 1.0f / std::sqrt(static_cast<float>(p->head_dim));
+}
+
+// Largest number of allowed key blocks of any query block (window x causal layers).
+int64_t max_candidates(const lcsa_params *p, const lcsa_kv_cache *c) {
+    auto span = [&](int n) -> int64_t {
+        if (p->local_range <= 0) return n;
+        if (p->local_mode == 0) return n <= p->local_range ? n : p->local_range;
+        return std::min<int64_t>(n, p->local_range);  // truncated: at most r along an axis
+    };
+    return static_cast<int64_t>(c->count) * span(p->grid_h) * span(p->grid_w);
+}
+
+// Rank-4 map over a token-layout bf16 tensor [H*T][8gh][8gw][128] with a
+// (64 dims, 8, 8, 2 frames) box and 128-byte swizzle: one box pair is one
+// (2,8,8) window block, so the partition is done by the copy engine.
+bool make_token_map(CUtensorMap *m, const void *base, int64_t frames, int tok_h, int tok_w) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(tok_w),
+                                static_cast<cuuint64_t>(tok_h), static_cast<cuuint64_t>(frames)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHeadDim) * 2,
+                                   static_cast<cuuint64_t>(kHeadDim) * 2 * tok_w,
+                                   static_cast<cuuint64_t>(kHeadDim) * 2 * tok_w * tok_h};
+    const cuuint32_t box[4] = {64, 8, 8, 2};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Rank-2 map over a block-layout ring [rows][128] with a (64 dims, 128 rows) box.
+bool make_ring_map(CUtensorMap *m, const void *base, int64_t rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBlockTokens)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lcsa_version(void) { return 100; }
+
+const char *lcsa_status_string(int code) {
+    switch (code) {
+        case LCSA_OK: return "LCSA_OK";
+        case LCSA_ERR_INVALID_ARG: return "LCSA_ERR_INVALID_ARG";
+        case LCSA_ERR_UNSUPPORTED_DEVICE: return "LCSA_ERR_UNSUPPORTED_DEVICE";
+        case LCSA_ERR_CUDA: return "LCSA_ERR_CUDA";
+        case LCSA_ERR_TIMEOUT: return "LCSA_ERR_TIMEOUT";
+        case LCSA_ERR_BAD_INDEX: return "LCSA_ERR_BAD_INDEX";
+        case LCSA_ERR_TIMEOUT | LCSA_ERR_BAD_INDEX: return "LCSA_ERR_TIMEOUT|LCSA_ERR_BAD_INDEX";
+        default: return "LCSA_ERR_UNKNOWN";
+    }
+}
+
+int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok, int32_t n_layers,
+                      int32_t *d_status, void *stream) {
+    (void)d_status;  // the append kernel has no device-side failure mode
+    int rc = check_cache(cache);
+    if (rc != LCSA_OK) return rc;
+    if (!k_tok || !v_tok || !aligned16(k_tok) || !aligned16(v_tok)) return LCSA_ERR_INVALID_ARG;
+    if (n_layers < 1 || n_layers > cache->capacity || n_layers > lcsa::kMaxAppendLayers) return LCSA_ERR_INVALID_ARG;
+    if ((rc = check_device()) != LCSA_OK) return rc;
+
+    lcsa::AppendArgs a{};
+    a.k_tok = static_cast<const uint16_t *>(k_tok);
+    a.v_tok = static_cast<const uint16_t *>(v_tok);
+    a.k_cache = static_cast<uint16_t *>(cache->k);
+    a.v_cache = static_cast<uint16_t *>(cache->v);
+    a.kmean = cache->kmean;
+    a.heads = cache->heads;
+    a.grid_h = cache->grid_h;
+    a.grid_w = cache->grid_w;
+    a.nblk = cache->grid_h * cache->grid_w;
+    a.tok_h = 8 * cache->grid_h;
+    a.tok_w = 8 * cache->grid_w;
+    a.n_layers = n_layers;
+    int oldest = cache->oldest, count = cache->count;
+    for (int i = 0; i < n_layers; ++i) {
+        if (count < cache->capacity) {
+            a.slots[i] = (oldest + count) % cache->capacity;
+            ++count;
+        } else {  // ring full: the oldest layer is dropped and its slot reused
+            a.slots[i] = oldest;
+            oldest = (oldest + 1) % cache->capacity;
+        }
+    }
+    if (lcsa::launch_cache_append(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LCSA_ERR_CUDA;
+    cache->oldest = oldest;
+    cache->count = count;
+    return LCSA_OK;
+}
+
+int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache *cache, int32_t *kept_idx,
+                    int32_t *kept_cnt, float *scores_opt, float *qmean_opt, int32_t *d_status, void *stream) {
+    int rc = check_cache(cache);
+    if (rc != LCSA_OK) return rc;
+    if ((rc = check_params(p, cache)) != LCSA_OK) return rc;
+    if (!q_tok || !aligned16(q_tok) || !kept_idx || !kept_cnt) return LCSA_ERR_INVALID_ARG;
+    if (max_candidates(p, cache) > lcsa::kMaxCandidates) return LCSA_ERR_INVALID_ARG;
+    if ((rc = check_device()) != LCSA_OK) return rc;
+
+    lcsa::DraftArgs a{};
+    a.q = static_cast<const uint16_t *>(q_tok);
+    a.kmean = cache->kmean;
+    a.heads = p->heads;
+    a.grid_h = p->grid_h;
+    a.grid_w = p->grid_w;
+    a.nblk = p->grid_h * p->grid_w;
+    a.q_layers = p->q_layers;
+    a.tq = 2 * p->q_layers;
+    a.tok_h = 8 * p->grid_h;
+    a.tok_w = 8 * p->grid_w;
+    a.capacity = cache->capacity;
+    a.oldest = cache->oldest;
+    a.count = cache->count;
+    a.local_range = p->local_range;
+    a.local_mode = p->local_mode;
+    a.topk = p->topk;
+    a.scale = eff_scale(p);
+    a.kept_idx = kept_idx;
+    a.kept_cnt = kept_cnt;
+    a.scores = scores_opt;
+    a.qmean = qmean_opt;
+    a.status = d_status;
+    if (lcsa::launch_draft(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LCSA_ERR_CUDA;
+    return LCSA_OK;
+}
+
+int lcsa_attention(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache *cache, const int32_t *kept_idx,
+                   const int32_t *kept_cnt, void *out_tok, float *lse_opt, int32_t *d_status, void *stream) {
+    int rc = check_cache(cache);
+    if (rc != LCSA_OK) return rc;
+    if ((rc = check_params(p, cache)) != LCSA_OK) return rc;
+    if (!q_tok || !out_tok || !aligned16(q_tok) || !aligned16(out_tok) || !kept_idx || !kept_cnt)
+        return LCSA_ERR_INVALID_ARG;
+    if (q_tok == out_tok) return LCSA_ERR_INVALID_ARG;
+    if ((rc = check_device()) != LCSA_OK) return rc;
+
+    const int nblk = p->grid_h * p->grid_w;
+    const int64_t frames = static_cast<int64_t>(p->heads) * 2 * p->q_layers;
+    const int64_t rows = static_cast<int64_t>(cache->capacity) * cache->heads * nblk * kBlockTokens;
+    CUtensorMap tq, tk, tv, to;
+    if (!make_token_map(&tq, q_tok, frames, 8 * p->grid_h, 8 * p->grid_w) ||
+        !make_token_map(&to, out_tok, frames, 8 * p->grid_h, 8 * p->grid_w) || !make_ring_map(&tk, cache->k, rows) ||
+        !make_ring_map(&tv, cache->v, rows))
+        return LCSA_ERR_CUDA;
+
+    lcsa::AttnArgs a{};
+    a.heads = p->heads;
+    a.grid_h = p->grid_h;
+    a.grid_w = p->grid_w;
+    a.nblk = nblk;
+    a.q_layers = p->q_layers;
+    a.tq = 2 * p->q_layers;
+    a.tok_h = 8 * p->grid_h;
+    a.tok_w = 8 * p->grid_w;
+    a.n_key_blocks = cache->count * nblk;
+    a.capacity = cache->capacity;
+    a.oldest = cache->oldest;
+    a.topk = p->topk;
+    a.n_units = p->heads * p->q_layers * nblk;
+    a.scale_log2 = eff_scale(p) * 1.4426950408889634f;
+    a.kept_idx = kept_idx;
+    a.kept_cnt = kept_cnt;
+    a.lse = lse_opt;
+    a.status = d_status;
+    a.timeout_ns = lcsa::kWatchdogNs;
+    a.flags = p->flags;
+    if (lcsa::launch_attention(tq, tk, tv, to, a, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return LCSA_ERR_CUDA;
+    return LCSA_OK;
+}
+
+}  // extern "C"

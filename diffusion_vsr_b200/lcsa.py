@@ -1,0 +1,197 @@
+"""ctypes binding of ``liblcsa.so`` (declarations in ``include/lcsa.h``).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+the library.  Tensors are torch CUDA tensors, passed by data pointer on the
+current stream.  There is no CPU fallback: loading fails loudly when the
+library is missing.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+LCSA_OK = 0
+LCSA_ERR_INVALID_ARG = 1
+LCSA_ERR_UNSUPPORTED_DEVICE = 2
+LCSA_ERR_CUDA = 3
+LCSA_ERR_TIMEOUT = 4
+LCSA_ERR_BAD_INDEX = 8
+LCSA_FLAG_FORCE_TIMEOUT = 1
+LCSA_MAX_CANDIDATES = 4096
+
+EXPORTED_SYMBOLS = ("lcsa_cache_append", "lcsa_draft_mask", "lcsa_attention", "lcsa_status_string",
+                    "lcsa_version")
+
+
+class lcsa_params(ctypes.Structure):
+    _fields_ = [("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("grid_h", ctypes.c_int32),
+                ("grid_w", ctypes.c_int32), ("q_layers", ctypes.c_int32), ("local_range", ctypes.c_int32),
+                ("local_mode", ctypes.c_int32), ("topk", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("flags", ctypes.c_int32)]
+
+
+class lcsa_kv_cache(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("kmean", ctypes.c_void_p),
+                ("capacity", ctypes.c_int32), ("oldest", ctypes.c_int32), ("count", ctypes.c_int32),
+                ("heads", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32)]
+
+
+class LcsaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {status_string(code)} ({code})")
+        self.code = code
+
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load liblcsa.so (built in-tree by ``diffusion_vsr_b200.build``)."""
+    global _LIB
+    if _LIB is not None and path is None:
+        return _LIB
+    path = path or _build.LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(f"LCSA CUDA library not built: {path} is missing "
+                           "(run `python -m diffusion_vsr_b200.build`)")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER
+    vp = ctypes.c_void_p
+    lib.lcsa_cache_append.argtypes = [P(lcsa_kv_cache), vp, vp, ctypes.c_int32, vp, vp]
+    lib.lcsa_cache_append.restype = ctypes.c_int
+    lib.lcsa_draft_mask.argtypes = [P(lcsa_params), vp, P(lcsa_kv_cache), vp, vp, vp, vp, vp, vp]
+    lib.lcsa_draft_mask.restype = ctypes.c_int
+    lib.lcsa_attention.argtypes = [P(lcsa_params), vp, P(lcsa_kv_cache), vp, vp, vp, vp, vp, vp]
+    lib.lcsa_attention.restype = ctypes.c_int
+    lib.lcsa_status_string.argtypes = [ctypes.c_int]
+    lib.lcsa_status_string.restype = ctypes.c_char_p
+    lib.lcsa_version.argtypes = []
+    lib.lcsa_version.restype = ctypes.c_int
+    if path == _build.LIB_PATH:
+        _LIB = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().lcsa_status_string(int(code)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("LCSA tensors must live on the GPU")
+    if not t.is_contiguous():
+        raise ValueError("LCSA tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != LCSA_OK:
+        raise LcsaError(fn, rc)
+
+
+def make_params(heads: int, grid_h: int, grid_w: int, q_layers: int, topk: int, local_range: int = 11,
+                local_mode: int = 0, scale: float = 0.0, flags: int = 0) -> lcsa_params:
+    return lcsa_params(heads, 128, grid_h, grid_w, q_layers, local_range, local_mode, topk, scale, flags)
+
+
+@dataclass
+class KVCache:
+    """Caller-owned ring buffers (torch CUDA tensors) plus the C descriptor."""
+    k: torch.Tensor       # bf16 [capacity, H, nblk, 128, 128]
+    v: torch.Tensor
+    kmean: torch.Tensor   # fp32 [capacity, H, nblk, 128]
+    desc: lcsa_kv_cache
+
+    @classmethod
+    def allocate(cls, capacity: int, heads: int, grid_h: int, grid_w: int, device="cuda") -> "KVCache":
+        nblk = grid_h * grid_w
+        k = torch.empty((capacity, heads, nblk, 128, 128), dtype=torch.bfloat16, device=device)
+        v = torch.empty_like(k)
+        km = torch.empty((capacity, heads, nblk, 128), dtype=torch.float32, device=device)
+        desc = lcsa_kv_cache(k.data_ptr(), v.data_ptr(), km.data_ptr(), capacity, 0, 0, heads, grid_h, grid_w)
+        return cls(k, v, km, desc)
+
+    @property
+    def count(self) -> int:
+        return self.desc.count
+
+    @property
+    def oldest(self) -> int:
+        return self.desc.oldest
+
+    def slot_of_layer(self, layer: int) -> int:
+        return (self.desc.oldest + layer) % self.desc.capacity
+
+    def reset(self) -> None:
+        self.desc.oldest = 0
+        self.desc.count = 0
+
+
+def lcsa_cache_append(cache: KVCache, k_tok: torch.Tensor, v_tok: torch.Tensor, n_layers: Optional[int] = None,
+                      d_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    if n_layers is None:
+        n_layers = k_tok.shape[1] // 2
+    rc = load_library().lcsa_cache_append(ctypes.byref(cache.desc), _ptr(k_tok), _ptr(v_tok), n_layers,
+                                          _ptr(d_status), _stream(stream))
+    _check("lcsa_cache_append", rc)
+
+
+def lcsa_draft_mask(params: lcsa_params, q_tok: torch.Tensor, cache: KVCache, kept_idx: torch.Tensor,
+                    kept_cnt: torch.Tensor, scores: Optional[torch.Tensor] = None,
+                    qmean: Optional[torch.Tensor] = None, d_status: Optional[torch.Tensor] = None,
+                    stream=None) -> None:
+    rc = load_library().lcsa_draft_mask(ctypes.byref(params), _ptr(q_tok), ctypes.byref(cache.desc),
+                                        _ptr(kept_idx), _ptr(kept_cnt), _ptr(scores), _ptr(qmean),
+                                        _ptr(d_status), _stream(stream))
+    _check("lcsa_draft_mask", rc)
+
+
+def lcsa_attention(params: lcsa_params, q_tok: torch.Tensor, cache: KVCache, kept_idx: torch.Tensor,
+                   kept_cnt: torch.Tensor, out_tok: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                   d_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    rc = load_library().lcsa_attention(ctypes.byref(params), _ptr(q_tok), ctypes.byref(cache.desc),
+                                       _ptr(kept_idx), _ptr(kept_cnt), _ptr(out_tok), _ptr(lse),
+                                       _ptr(d_status), _stream(stream))
+    _check("lcsa_attention", rc)
+
+
+class LcsaLayer:
+    """One LCSA attention layer of a streaming DiT: cache + draft + attention.
+
+    Owns the ring and the per-step buffers; ``step`` appends the chunk's k/v,
+    builds the draft mask and runs the block-sparse attention, all on the
+    current stream.
+    """
+
+    def __init__(self, heads: int, grid_h: int, grid_w: int, q_layers: int, kv_len: int, topk: int,
+                 local_range: int = 11, local_mode: int = 0, device="cuda"):
+        self.params = make_params(heads, grid_h, grid_w, q_layers, topk, local_range, local_mode)
+        self.cache = KVCache.allocate(kv_len + q_layers, heads, grid_h, grid_w, device)
+        nq = q_layers * grid_h * grid_w
+        self.kept_idx = torch.empty((heads, nq, topk), dtype=torch.int32, device=device)
+        self.kept_cnt = torch.empty((heads, nq), dtype=torch.int32, device=device)
+        self.status = torch.zeros((1,), dtype=torch.int32, device=device)
+
+    def append(self, k_tok: torch.Tensor, v_tok: torch.Tensor) -> None:
+        lcsa_cache_append(self.cache, k_tok, v_tok, d_status=self.status)
+
+    def step(self, q_tok: torch.Tensor, k_tok: torch.Tensor, v_tok: torch.Tensor, out_tok: torch.Tensor,
+             lse: Optional[torch.Tensor] = None) -> None:
+        lcsa_cache_append(self.cache, k_tok, v_tok, d_status=self.status)
+        lcsa_draft_mask(self.params, q_tok, self.cache, self.kept_idx, self.kept_cnt, d_status=self.status)
+        lcsa_attention(self.params, q_tok, self.cache, self.kept_idx, self.kept_cnt, out_tok, lse,
+                       d_status=self.status)

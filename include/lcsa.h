@@ -1,0 +1,159 @@
+/*
+ * lcsa.h - C ABI of the B200 (sm_100a) locality-constrained block-sparse
+ * causal attention (LCSA) hot path of FlashVSR's one-step streaming DiT.
+ *
+ * Sources of the operations (page title, section):
+ *  - "FlashVSR 是怎么工作的" (vsr-hover-compare learn.html), 2.2 LCSA:
+ *    WindowPartition3D into (2,8,8) blocks, local block mask (default
+ *    local_range 11), block mean pooling, draft scores q.k/sqrt(D), -inf
+ *    outside the mask, top-k, block_sparse_attn_func over the kept pairs.
+ *  - same page, 2.3 streaming + KV cache: keep the newest kv_len block-layers,
+ *    drop the oldest one per step.
+ *  - reading notes "FlashVSR: Towards Real-time Diffusion-Based Streaming
+ *    Video Super Resolution", 关键设计 1 (causal mask), 2 (block-sparse
+ *    attention on top-k 128x128 block pairs), 3 (local window, the
+ *    Boundary-Preserved and Boundary-Truncated rules).
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *    allocated and owned by the caller; the library never allocates or frees
+ *    device memory.  Tensor pointers must be 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*,
+ *    NULL = legacy default stream).
+ *  - Return value: LCSA_OK, or an LCSA_ERR_* code for a synchronous argument
+ *    or launch error; nothing is enqueued when an error is returned.
+ *  - Device-side errors (a watchdog that expired, an out-of-range kept index)
+ *    are OR-ed into *d_status (a device int32 the caller zeroes and reads
+ *    after synchronising); d_status may be NULL to ignore them.
+ *  - Token layout of q/k/v/out: bf16 [heads][frames][8*grid_h][8*grid_w][128],
+ *    frames = 2 per block-layer.  Block b of a layer is (by, bx) =
+ *    (b / grid_w, b % grid_w); token n of a block is
+ *    (t, y, x) = (n / 64, (n / 8) % 8, n % 8) (row-major in (t, y, x)).
+ *  - Key-block indices are LOGICAL: j = layer * grid_h*grid_w + b, layer 0
+ *    being the oldest resident layer of the cache.
+ *  - Only compute capability 10.0 (B200) is supported.
+ */
+#ifndef LCSA_H
+#define LCSA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum lcsa_status {
+    LCSA_OK = 0,
+    LCSA_ERR_INVALID_ARG = 1,
+    LCSA_ERR_UNSUPPORTED_DEVICE = 2,
+    LCSA_ERR_CUDA = 3,
+    /* device status bits (OR-ed into *d_status) */
+    LCSA_ERR_TIMEOUT = 4,    /* a bounded wait inside a kernel gave up */
+    LCSA_ERR_BAD_INDEX = 8   /* a kept index / count was out of range */
+};
+
+/* lcsa_params.flags */
+#define LCSA_FLAG_FORCE_TIMEOUT 1 /* test hook: the first consumer wait of
+                                     lcsa_attention gives up at once */
+
+#define LCSA_HEAD_DIM 128
+#define LCSA_BLOCK_TOKENS 128
+#define LCSA_MAX_CANDIDATES 4096 /* allowed key blocks per query block */
+
+typedef struct lcsa_params {
+    int32_t heads;       /* H >= 1 */
+    int32_t head_dim;    /* must be 128 */
+    int32_t grid_h;      /* blocks per latent frame along y (tokens / 8) */
+    int32_t grid_w;      /* blocks per latent frame along x (tokens / 8) */
+    int32_t q_layers;    /* query block-layers: the newest q_layers of the cache */
+    int32_t local_range; /* window side in blocks (odd, e.g. 11); <= 0: no window */
+    int32_t local_mode;  /* 0 Boundary-Preserved (window shifted inside the
+                            grid), 1 Boundary-Truncated (|i-j| <= range/2) */
+    int32_t topk;        /* kept key blocks per query block, >= 1; also the
+                            row stride of kept_idx */
+    float scale;         /* softmax scale; 0 -> 1/sqrt(head_dim) */
+    int32_t flags;       /* LCSA_FLAG_*; 0 in normal use */
+} lcsa_params;
+
+/* Ring of block-layers, caller-owned device buffers:
+ *   k, v   bf16 [capacity][heads][grid_h*grid_w][128 tokens][128]
+ *   kmean  fp32 [capacity][heads][grid_h*grid_w][128]  (block means of k)
+ * Slot of logical layer L: (oldest + L) % capacity.  `oldest` and `count`
+ * are host-side state updated by lcsa_cache_append; start from 0, 0. */
+typedef struct lcsa_kv_cache {
+    void *k;
+    void *v;
+    float *kmean;
+    int32_t capacity; /* kv_len + layers of one step */
+    int32_t oldest;
+    int32_t count;
+    int32_t heads;
+    int32_t grid_h;
+    int32_t grid_w;
+} lcsa_kv_cache;
+
+/*
+ * lcsa_cache_append - append n_layers block-layers of keys and values
+ * (learn.html 2.3: the cache keeps the newest layers and drops the oldest).
+ *   k_tok, v_tok: bf16 token layout [heads][2*n_layers][8*grid_h][8*grid_w][128].
+ * Each layer is written in block layout (partition of learn.html 2.2) into
+ * the next ring slot, together with its fp32 block means of k; when the
+ * ring is full the oldest layer's slot is overwritten and `oldest` advances.
+ * Updates cache->oldest/count on the host when the copy is enqueued, so calls
+ * on one cache must be serialised by the caller.  1 <= n_layers <= capacity.
+ */
+int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok,
+                      int32_t n_layers, int32_t *d_status, void *stream);
+
+/*
+ * lcsa_draft_mask - the draft mask of learn.html 2.2, one row per
+ * (head, query block).  Query block i of layer ql sits at key layer
+ * count - q_layers + ql.  Steps: fp32 block mean of q (fixed-order sum,
+ * times 1/128); for every key block j allowed by the local window (same
+ * spatial window on every layer, rule per local_mode) and by block causality
+ * (key layer <= query layer): s = mean_q . kmean_j * scale, in fp32; keep the
+ * min(topk, allowed) largest s, ties to the lower j.
+ *   q_tok      bf16 token layout [heads][2*q_layers][8*grid_h][8*grid_w][128]
+ *   kept_idx   int32 [heads][q_layers*grid_h*grid_w][topk]: kept j ascending,
+ *              padded with -1
+ *   kept_cnt   int32 [heads][q_layers*grid_h*grid_w]
+ *   scores_opt fp32 [heads][Nq][count*grid_h*grid_w] or NULL: s for allowed
+ *              pairs, -inf elsewhere
+ *   qmean_opt  fp32 [heads][Nq][128] or NULL: the q block means
+ * Allowed candidates per row must not exceed LCSA_MAX_CANDIDATES.
+ */
+int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache *cache,
+                    int32_t *kept_idx, int32_t *kept_cnt, float *scores_opt,
+                    float *qmean_opt, int32_t *d_status, void *stream);
+
+/*
+ * lcsa_attention - block_sparse_attn_func of learn.html 2.2 (reading notes
+ * 关键设计 2): for every query token of block i, exact
+ * softmax(q k^T * scale) V over the 128 tokens of each kept key block of row
+ * (h, i) and nothing else; online softmax with fp32 accumulation, bf16
+ * tensor-core products.
+ *   q_tok    bf16 token layout [heads][2*q_layers][8*grid_h][8*grid_w][128]
+ *   kept_idx int32 [heads][Nq][topk], kept_cnt int32 [heads][Nq]: the first
+ *            kept_cnt entries of a row are used (any order, no duplicates)
+ *   out_tok  bf16, same layout as q_tok (written; may not alias q_tok)
+ *   lse_opt  fp32 [heads][2*q_layers][8*grid_h][8*grid_w] or NULL: natural
+ *            log of the softmax denominator of each query token
+ * A row with kept_cnt == 0 gets zeros (lse -inf).  A kept index outside
+ * [0, count*grid_h*grid_w) or a count outside [0, topk] sets
+ * LCSA_ERR_BAD_INDEX and the row is written as if it kept nothing.
+ */
+int lcsa_attention(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache *cache,
+                   const int32_t *kept_idx, const int32_t *kept_cnt, void *out_tok,
+                   float *lse_opt, int32_t *d_status, void *stream);
+
+/* Human-readable name of a status code or of a device status word. */
+const char *lcsa_status_string(int code);
+
+/* Library ABI version (major * 100 + minor). */
+int lcsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LCSA_H */

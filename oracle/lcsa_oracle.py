@@ -177,12 +177,13 @@ def sparse_attention_row(q_blk: np.ndarray, k_blocks: np.ndarray, v_blocks: np.n
     probability matrix when asked.  An empty kept list gives zeros and -inf.
     """
     kept = list(kept)
+    q_blk = np.asarray(q_blk, dtype=np.float64)
     if not kept:
         out = np.zeros_like(q_blk, dtype=np.float64)
         lse = np.full(q_blk.shape[0], -np.inf)
         return (out, lse, None) if return_probs else (out, lse)
-    keys = k_blocks[kept].reshape(-1, k_blocks.shape[-1])
-    vals = v_blocks[kept].reshape(-1, v_blocks.shape[-1])
+    keys = k_blocks[kept].reshape(-1, k_blocks.shape[-1]).astype(np.float64)
+    vals = v_blocks[kept].reshape(-1, v_blocks.shape[-1]).astype(np.float64)
     logits = (q_blk @ keys.T) * scale
     m = logits.max(axis=1, keepdims=True)
     p = np.exp(logits - m)
@@ -290,7 +291,7 @@ def lcsa_step(q_tok: np.ndarray, cache: KVCacheModel, grid_h: int, grid_w: int, 
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     qb = partition(q_tok)
-    kb, vb = cache.keys()
+    kb, vb = cache.keys()  # any float dtype holding exact values; arithmetic below is fp64
     k_layers = cache.count
     mq = block_means(qb)
     mk = block_means(kb)

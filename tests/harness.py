@@ -1,0 +1,160 @@
+"""Test-side glue: runs a workload through the CUDA library and the oracle.
+
+Test infrastructure (imports the oracle).  The CUDA side goes through the
+ctypes binding of the C ABI only.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Tuple
+
+import numpy as np
+import torch
+
+from diffusion_vsr_b200 import workloads as W
+from oracle import lcsa_oracle as O
+
+MODES = {0: "preserved", 1: "truncated"}
+ATOL_OUT = 2e-2      # max-abs error of bf16 outputs against the fp64 oracle
+RTOL_L2_OUT = 5e-3   # relative L2 error of bf16 outputs against the fp64 oracle
+NEAR_TIE_REL = 1e-5
+
+
+def f32(t: torch.Tensor) -> np.ndarray:
+    """Exact fp32 copy of a bf16 tensor as numpy (the oracle upcasts to fp64)."""
+    return t.to(torch.float32).cpu().numpy()
+
+
+def rel_l2(a: np.ndarray, b: np.ndarray) -> float:
+    return float(np.linalg.norm((a - b).ravel()) / max(np.linalg.norm(b.ravel()), 1e-300))
+
+
+def compare_outputs(gpu_blocks: np.ndarray, ref_blocks: np.ndarray) -> Tuple[float, float]:
+    err = np.abs(gpu_blocks - ref_blocks)
+    return float(err.max()), rel_l2(gpu_blocks, ref_blocks)
+
+
+def sample_rows(H: int, Nq: int, n: int, seed: int) -> List[Tuple[int, int]]:
+    rng = np.random.default_rng(seed)
+    rows = {(0, 0), (H - 1, Nq - 1), (0, Nq - 1), (H - 1, 0)}
+    while len(rows) < min(n, H * Nq):
+        rows.add((int(rng.integers(H)), int(rng.integers(Nq))))
+    return sorted(rows)
+
+
+@dataclass
+class StepResult:
+    position: int
+    oracle: Dict[str, np.ndarray]
+    gpu_kept: np.ndarray
+    gpu_cnt: np.ndarray
+    gpu_scores: np.ndarray
+    gpu_qmean: np.ndarray
+    out_pipeline: np.ndarray      # GPU output with the GPU's own mask, block layout fp32
+    out_oracle_mask: np.ndarray   # GPU output fed the oracle's mask, block layout fp32
+    lse_oracle_mask: np.ndarray   # [H, Nq, 128]
+    rows: List[Tuple[int, int]]
+    exempt: np.ndarray
+    status: int
+    ring_ok: Optional[bool] = None
+    kmean_err: Optional[float] = None
+
+
+def run_stream(w: W.Workload, n_steps: Optional[int] = None, n_rows: Optional[int] = None,
+               check_ring: bool = False, seed_rows: int = 0) -> List[StepResult]:
+    """Run prefill + steps of ``w`` on the GPU and the oracle side by side."""
+    from diffusion_vsr_b200 import lcsa as L
+
+    dev = torch.device("cuda")
+    layer = L.LcsaLayer(w.heads, w.grid_h, w.grid_w, w.q_layers, w.kv_len, w.topk, w.local_range,
+                        w.local_mode, device=dev)
+    ocache = O.KVCacheModel(w.capacity)
+    prefill, steps = W.stream_plan(w)
+    for p in prefill:
+        _, k, v = W.gen_layers(w, p, 1, "kv")
+        layer.append(k.to(dev), v.to(dev))
+        ocache.append(f32(k), f32(v))
+    Nq = w.n_query_blocks
+    results = []
+    for p in steps[: (n_steps or len(steps))]:
+        q, k, v = W.gen_layers(w, p, w.q_layers)
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        L.lcsa_cache_append(layer.cache, kd, vd, d_status=layer.status)
+        ocache.append(f32(k), f32(v))
+        ring_ok = None
+        kmean_err = None
+        if check_ring:
+            ring_ok, kmean_err = ring_matches(layer.cache, ocache)
+        Nk = layer.cache.count * w.blocks_per_layer
+        scores = torch.empty((w.heads, Nq, Nk), dtype=torch.float32, device=dev)
+        qmean = torch.empty((w.heads, Nq, 128), dtype=torch.float32, device=dev)
+        L.lcsa_draft_mask(layer.params, qd, layer.cache, layer.kept_idx, layer.kept_cnt, scores, qmean,
+                          d_status=layer.status)
+        out_p = torch.empty_like(qd)
+        L.lcsa_attention(layer.params, qd, layer.cache, layer.kept_idx, layer.kept_cnt, out_p,
+                         d_status=layer.status)
+        # oracle draft + selection on every row; attention on sampled rows
+        rows = None if n_rows is None else sample_rows(w.heads, Nq, n_rows, seed_rows + p)
+        ref = O.lcsa_step(f32(q), ocache, w.grid_h, w.grid_w, w.topk, w.local_range, MODES[w.local_mode],
+                          rows=rows if rows is not None else [(h, i) for h in range(w.heads) for i in range(Nq)])
+        kept_o = torch.from_numpy(ref["kept_idx"]).to(dev)
+        cnt_o = torch.from_numpy(ref["kept_cnt"]).to(dev)
+        out_o = torch.empty_like(qd)
+        lse_o = torch.empty(qd.shape[:4], dtype=torch.float32, device=dev)
+        L.lcsa_attention(layer.params, qd, layer.cache, kept_o, cnt_o, out_o, lse_o, d_status=layer.status)
+        torch.cuda.synchronize()
+        exempt = O.near_tie_rows(ref["scores"], ref["allowed"], ref["mq"], ref["mk"], w.topk, NEAR_TIE_REL)
+        results.append(StepResult(
+            position=p, oracle=ref,
+            gpu_kept=layer.kept_idx.cpu().numpy(), gpu_cnt=layer.kept_cnt.cpu().numpy(),
+            gpu_scores=scores.cpu().numpy(), gpu_qmean=qmean.cpu().numpy(),
+            out_pipeline=O.partition(f32(out_p)), out_oracle_mask=O.partition(f32(out_o)),
+            lse_oracle_mask=O.partition(lse_o.cpu().numpy()[..., None])[..., 0],
+            rows=rows if rows is not None else [(h, i) for h in range(w.heads) for i in range(Nq)],
+            exempt=exempt, status=int(layer.status.item()), ring_ok=ring_ok, kmean_err=kmean_err))
+    return results
+
+
+def ring_matches(cache, ocache: O.KVCacheModel) -> Tuple[bool, float]:
+    """Ring slots hold exactly the oracle's partitioned layers, oldest first."""
+    ok = cache.count == ocache.count
+    worst = 0.0
+    for layer_i, (kb, vb) in enumerate(ocache.layers):
+        slot = cache.slot_of_layer(layer_i)
+        gk = cache.k[slot].to(torch.float32).cpu().numpy()
+        gv = cache.v[slot].to(torch.float32).cpu().numpy()
+        ok &= np.array_equal(gk, kb) and np.array_equal(gv, vb)
+        gm = cache.kmean[slot].cpu().numpy().astype(np.float64)
+        om = O.block_means(kb)
+        worst = max(worst, float(np.max(np.abs(gm - om) / (np.abs(kb).mean(axis=2) + 1e-30))))
+    return bool(ok), worst
+
+
+def check_mask(res: StepResult, w: W.Workload) -> Tuple[int, int, int]:
+    """(rows compared bit-exactly, exempt rows, mismatching rows)."""
+    ref = res.oracle
+    H, Nq = ref["kept_cnt"].shape
+    bad = 0
+    exact = 0
+    n_exempt = 0
+    for h in range(H):
+        for i in range(Nq):
+            g = res.gpu_kept[h, i, :res.gpu_cnt[h, i]]
+            if res.exempt[h, i]:
+                n_exempt += 1
+                sr = ref["scores"][h, i]
+                cand = np.nonzero(ref["allowed"][i])[0]
+                # same scale as the exemption rule: |mq| |mk| / sqrt(D) bounds sum |mq_d mk_d| / sqrt(D)
+                mag = np.linalg.norm(ref["mq"][h, i]) * np.linalg.norm(ref["mk"][h, cand], axis=1).max()
+                tol = NEAR_TIE_REL * mag / math.sqrt(ref["mq"].shape[-1])
+                if not O.valid_topk(g, sr, ref["allowed"][i], w.topk, tol):
+                    bad += 1
+                continue
+            exact += 1
+            o = ref["kept_idx"][h, i, :ref["kept_cnt"][h, i]]
+            if res.gpu_cnt[h, i] != ref["kept_cnt"][h, i] or not np.array_equal(g, o) or \
+                    not np.all(res.gpu_kept[h, i, res.gpu_cnt[h, i]:] == -1):
+                bad += 1
+    return exact, n_exempt, bad

@@ -1,0 +1,221 @@
+"""GPU parity of the CUDA path against the fp64 oracle, through the C ABI.
+
+Acceptance: the kept block set is bit-exact except on near-tie rows (which
+must still be a valid top-k); outputs fed the oracle's own mask are within
+max-abs 2e-2 and relative L2 5e-3 of the fp64 oracle; the ring holds exactly
+the partitioned layers; block means within 1e-6 relative.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from diffusion_vsr_b200 import workloads as W
+from oracle import lcsa_oracle as O
+from tests import harness as Hn
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    from diffusion_vsr_b200 import lcsa
+    return lcsa
+
+
+def _check_step(res, w, require_rows_exact=True):
+    ref = res.oracle
+    assert res.status == 0, _lib().status_string(res.status)
+    # q block means and fp32 draft scores against fp64
+    np.testing.assert_allclose(res.gpu_qmean, ref["mq"], rtol=1e-6, atol=1e-7)
+    allowed = ref["allowed"]
+    gs = res.gpu_scores
+    assert np.all(np.isneginf(gs[:, ~allowed]))
+    mag = (np.linalg.norm(ref["mq"], axis=-1)[:, :, None] * np.linalg.norm(ref["mk"], axis=-1)[:, None, :]
+           / math.sqrt(128))
+    err = np.abs(gs - ref["scores"])[:, allowed]
+    assert np.all(err <= 1e-5 * mag[:, allowed] + 1e-9)
+    # kept sets
+    exact, exempt, bad = Hn.check_mask(res, w)
+    assert bad == 0, f"{bad} rows differ ({exact} exact, {exempt} near-tie)"
+    if require_rows_exact:
+        assert exact > 0.9 * (exact + exempt)
+    # attention with the oracle's mask
+    hs, iis = zip(*res.rows)
+    g = res.out_oracle_mask[list(hs), list(iis)]
+    o = ref["out_blocks"][list(hs), list(iis)]
+    mx, rl2 = Hn.compare_outputs(g, o)
+    assert mx <= Hn.ATOL_OUT and rl2 <= Hn.RTOL_L2_OUT, (mx, rl2)
+    lse_g = res.lse_oracle_mask[list(hs), list(iis)]
+    lse_o = ref["lse_blocks"][list(hs), list(iis)]
+    assert np.max(np.abs(lse_g - lse_o)) <= 2e-3
+    # the full pipeline equals the oracle-mask run bit for bit where the masks agree
+    same = np.all(res.gpu_kept == ref["kept_idx"], axis=-1) & (res.gpu_cnt == ref["kept_cnt"])
+    assert np.array_equal(res.out_pipeline[same], res.out_oracle_mask[same])
+    return mx, rl2
+
+
+def test_tiny_full_parity_with_ring():
+    w = W.WORKLOADS["tiny"]
+    (res,) = Hn.run_stream(w, check_ring=True)
+    assert res.ring_ok and res.kmean_err <= 1e-6
+    _check_step(res, w)
+
+
+def test_tiny_dense_equivalence_when_everything_is_kept():
+    # topk >= allowed and the window covers the grid: the CUDA path must equal
+    # dense block-causal attention.
+    w = W.WORKLOADS["tiny"].with_topk(32)
+    (res,) = Hn.run_stream(w)
+    assert np.all(res.gpu_cnt[:, :16] == 16) and np.all(res.gpu_cnt[:, 16:] == 32)
+    _check_step(res, w)
+    q, k, v = W.gen_layers(w, 0, w.q_layers)
+    dense = O.dense_block_causal_attention(Hn.f32(q), Hn.f32(k), Hn.f32(v), 1 / math.sqrt(128))
+    mx, rl2 = Hn.compare_outputs(res.out_pipeline, O.partition(dense))
+    assert mx <= Hn.ATOL_OUT and rl2 <= Hn.RTOL_L2_OUT
+
+
+def test_768x1280_full_parity():
+    w = W.WORKLOADS["768x1280"]
+    (res,) = Hn.run_stream(w, check_ring=True)
+    assert res.ring_ok and res.kmean_err <= 1e-6
+    _check_step(res, w)
+
+
+def test_768x1408_streaming_eight_chunks():
+    w = W.WORKLOADS["768x1408"]
+    results = Hn.run_stream(w, n_rows=24, check_ring=True)
+    assert len(results) == 8
+    for res in results:
+        assert res.ring_ok and res.kmean_err <= 1e-6
+        _check_step(res, w)
+
+
+def test_1536x2688_sampled():
+    w = W.WORKLOADS["1536x2688"]
+    for res in Hn.run_stream(w, n_steps=2, n_rows=16, check_ring=True):
+        assert res.ring_ok
+        _check_step(res, w)
+
+
+@pytest.mark.parametrize("topk", W.FOURK_TOPK_SWEEP)
+def test_4k_sampled(topk):
+    w = W.WORKLOADS["4k"].with_topk(topk)
+    for res in Hn.run_stream(w, n_steps=1, n_rows=12):
+        _check_step(res, w)
+
+
+def test_truncated_window_ragged_counts():
+    # Boundary-Truncated with a 5-block window: edge rows allow fewer blocks
+    # than topk, so kept counts are ragged.
+    import dataclasses
+    w = dataclasses.replace(W.WORKLOADS["768x1280"], local_mode=1, local_range=5, topk=40, heads=4)
+    (res,) = Hn.run_stream(w)
+    assert len(np.unique(res.gpu_cnt)) > 1 and res.gpu_cnt.min() < 40
+    _check_step(res, w)
+
+
+def test_deterministic_byte_identical():
+    w = W.WORKLOADS["768x1280"]
+    a = Hn.run_stream(w, n_rows=4)[0]
+    b = Hn.run_stream(w, n_rows=4)[0]
+    assert np.array_equal(a.gpu_kept, b.gpu_kept)
+    assert np.array_equal(a.gpu_scores, b.gpu_scores)
+    assert np.array_equal(a.out_pipeline, b.out_pipeline)
+
+
+# ------------------------------------------------------------------ edge cases
+
+def _tiny_setup(topk=8):
+    L = _lib()
+    w = W.WORKLOADS["tiny"]
+    q, k, v = [t.cuda() for t in W.gen_layers(w, 0, w.q_layers)]
+    layer = L.LcsaLayer(w.heads, w.grid_h, w.grid_w, w.q_layers, w.kv_len, topk, device="cuda")
+    layer.append(k, v)
+    return L, w, q, k, v, layer
+
+
+def test_zero_and_single_tile_rows():
+    L, w, q, k, v, layer = _tiny_setup(topk=4)
+    Nq = w.n_query_blocks
+    kept = torch.full((w.heads, Nq, 4), -1, dtype=torch.int32)
+    cnt = torch.zeros((w.heads, Nq), dtype=torch.int32)
+    rng = np.random.default_rng(3)
+    for h in range(w.heads):
+        for i in range(Nq):
+            c = int(rng.integers(0, 5))  # 0..4 tiles, ragged
+            sel = np.sort(rng.choice(32, size=c, replace=False))
+            kept[h, i, :c] = torch.from_numpy(sel.astype(np.int32))
+            cnt[h, i] = c
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:4], dtype=torch.float32, device="cuda")
+    L.lcsa_attention(layer.params, q, layer.cache, kept.cuda(), cnt.cuda(), out, lse, d_status=layer.status)
+    torch.cuda.synchronize()
+    assert layer.status.item() == 0
+    qb = O.partition(Hn.f32(q))
+    kb = O.partition(Hn.f32(k))
+    vb = O.partition(Hn.f32(v))
+    ob = O.partition(Hn.f32(out))
+    lb = O.partition(lse.cpu().numpy()[..., None])[..., 0]
+    for h in range(w.heads):
+        for i in range(Nq):
+            ro, rl = O.sparse_attention_row(qb[h, i], kb[h], vb[h], kept[h, i, :cnt[h, i]].numpy(), 1 / math.sqrt(128))
+            if cnt[h, i] == 0:
+                assert np.all(ob[h, i] == 0) and np.all(np.isneginf(lb[h, i]))
+            else:
+                assert np.max(np.abs(ob[h, i] - ro)) <= Hn.ATOL_OUT
+                assert np.max(np.abs(lb[h, i] - rl)) <= 2e-3
+
+
+def test_bad_kept_index_is_reported_and_row_zeroed():
+    L, w, q, k, v, layer = _tiny_setup(topk=8)
+    L.lcsa_draft_mask(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt)
+    good = torch.empty_like(q)
+    L.lcsa_attention(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, good)
+    kept = layer.kept_idx.clone()
+    cnt = layer.kept_cnt.clone()
+    kept[1, 5, 0] = 32          # one past the last key block
+    cnt[0, 7] = 9               # more than topk
+    out = torch.empty_like(q)
+    layer.status.zero_()
+    L.lcsa_attention(layer.params, q, layer.cache, kept, cnt, out, d_status=layer.status)
+    torch.cuda.synchronize()
+    assert layer.status.item() & L.LCSA_ERR_BAD_INDEX
+    ob, gb = O.partition(Hn.f32(out)), O.partition(Hn.f32(good))
+    assert np.all(ob[1, 5] == 0) and np.all(ob[0, 7] == 0)
+    mask = np.ones(ob.shape[:2], dtype=bool)
+    mask[1, 5] = mask[0, 7] = False
+    assert np.array_equal(ob[mask], gb[mask])
+
+
+def test_forced_watchdog_expiry_reports_timeout_and_context_survives():
+    L, w, q, k, v, layer = _tiny_setup(topk=8)
+    L.lcsa_draft_mask(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt)
+    ref = torch.empty_like(q)
+    L.lcsa_attention(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, ref)
+    p = L.make_params(w.heads, w.grid_h, w.grid_w, w.q_layers, 8, flags=L.LCSA_FLAG_FORCE_TIMEOUT)
+    out = torch.empty_like(q)
+    layer.status.zero_()
+    L.lcsa_attention(p, q, layer.cache, layer.kept_idx, layer.kept_cnt, out, d_status=layer.status)
+    torch.cuda.synchronize()
+    assert layer.status.item() & L.LCSA_ERR_TIMEOUT
+    # the context is still usable and gives the same result as before
+    again = torch.empty_like(q)
+    L.lcsa_attention(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, again)
+    torch.cuda.synchronize()
+    assert torch.equal(again, ref)
+
+
+def test_invalid_arguments_are_rejected():
+    L, w, q, k, v, layer = _tiny_setup()
+    out = torch.empty_like(q)
+    bad = L.make_params(w.heads, w.grid_h, w.grid_w, w.q_layers, 8, local_range=4)  # even range
+    with pytest.raises(L.LcsaError) as e:
+        L.lcsa_attention(bad, q, layer.cache, layer.kept_idx, layer.kept_cnt, out)
+    assert e.value.code == L.LCSA_ERR_INVALID_ARG
+    too_many = L.make_params(w.heads, w.grid_h, w.grid_w, 3, 8)  # more query layers than cached
+    with pytest.raises(L.LcsaError):
+        L.lcsa_draft_mask(too_many, q, layer.cache, layer.kept_idx, layer.kept_cnt)
+    with pytest.raises(L.LcsaError):
+        L.lcsa_attention(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, q)  # aliasing
