@@ -148,6 +148,20 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Largest value of ``x`` over all ranks (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world: int, flops_per_rank_step: float, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's work divided by the slowest rank's time."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def run_lcsa(args, rank: int, world: int, local_rank: int):
@@ -212,13 +226,10 @@ def run_lcsa(args, rank: int, world: int, local_rank: int):
     t_append = [e[0].elapsed_time(e[1]) for e in evs]
     t_draft = [e[1].elapsed_time(e[2]) for e in evs]
     t_attn = [e[2].elapsed_time(e[3]) for e in evs]
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_step = total_ms / args.steps
     step_flops = kept_tiles * flop_tile
-    value = world * step_flops / (ms_step * 1e-3) / 1e12
+    value = aggregate_tflops(world, step_flops, ms_step)
 
     pk = peaks()
     attn_ms = statistics.mean(t_attn)
@@ -313,14 +324,10 @@ def run_e2e(args, L, layer, host, dev, stream, step_flops, world):
         e2e_step(i)
     t1.record(stream)
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, dev)
     h2d = sum(t.numel() * t.element_size() for t in pinned[0])
     d2h = out_host.numel() * out_host.element_size()
-    return {"value": round(world * step_flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    return {"value": round(aggregate_tflops(world, step_flops, ms), 3), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
 
 

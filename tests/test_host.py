@@ -1,0 +1,133 @@
+"""CPU-only checks of the host side: the C library loads and exports every
+symbol the header declares, host-side argument validation (no GPU call is
+made on those paths), and the multi-rank reduction of the benchmark."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from diffusion_vsr_b200 import build as B
+from diffusion_vsr_b200 import lcsa as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    with open(os.path.join(ROOT, "include", "lcsa.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(lcsa_\w+)\s*\(", text, re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load_library()
+
+
+def test_header_declares_the_three_hot_path_calls():
+    fns = header_functions()
+    for name in ("lcsa_cache_append", "lcsa_draft_mask", "lcsa_attention"):
+        assert name in fns
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    assert set(L.EXPORTED_SYMBOLS) <= set(header_functions())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.lcsa_version() == 100
+    assert L.status_string(L.LCSA_OK) == "LCSA_OK"
+    assert L.status_string(L.LCSA_ERR_TIMEOUT) == "LCSA_ERR_TIMEOUT"
+    assert L.status_string(L.LCSA_ERR_BAD_INDEX | L.LCSA_ERR_TIMEOUT).startswith("LCSA_ERR_TIMEOUT|")
+
+
+def _fake_cache(**kw):
+    c = L.lcsa_kv_cache(0x10000, 0x20000, 0x30000, 4, 0, 4, 2, 4, 4)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def test_cache_append_rejects_bad_arguments_without_touching_the_gpu(lib):
+    c = _fake_cache()
+    assert lib.lcsa_cache_append(None, 0x40000, 0x50000, 1, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), None, 0x50000, 1, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40008, 0x50000, 1, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 5, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    bad = _fake_cache(count=5)
+    assert lib.lcsa_cache_append(ctypes.byref(bad), 0x40000, 0x50000, 1, None, None) == L.LCSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("field,value", [("head_dim", 64), ("topk", 0), ("local_range", 4), ("local_mode", 2),
+                                         ("q_layers", 5), ("heads", 3), ("scale", -1.0), ("grid_w", 5)])
+def test_draft_and_attention_reject_bad_params(lib, field, value):
+    p = L.make_params(2, 4, 4, 1, 8)
+    setattr(p, field, value)
+    c = _fake_cache()
+    z = ctypes.c_void_p(0x60000)
+    assert lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None) == \
+        L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_attention(ctypes.byref(p), z, ctypes.byref(c), z, z, ctypes.c_void_p(0x70000), None, None,
+                              None) == L.LCSA_ERR_INVALID_ARG
+
+
+def test_draft_rejects_too_many_candidates(lib):
+    # no window over a 64 x 64 block grid: 4096 per layer x 4 layers > 4096
+    p = L.make_params(1, 64, 64, 1, 8, local_range=0)
+    c = _fake_cache(heads=1, grid_h=64, grid_w=64)
+    z = ctypes.c_void_p(0x60000)
+    assert lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None) == \
+        L.LCSA_ERR_INVALID_ARG
+
+
+def test_attention_rejects_aliased_output(lib):
+    p = L.make_params(2, 4, 4, 1, 8)
+    c = _fake_cache()
+    z = ctypes.c_void_p(0x60000)
+    assert lib.lcsa_attention(ctypes.byref(p), z, ctypes.byref(c), z, z, z, None, None, None) == \
+        L.LCSA_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors():
+    with pytest.raises(ValueError):
+        L._ptr(torch.zeros(4))
+
+
+# ------------------------------------------------ multi-rank bench reduction
+
+def _rank_main(rank, world, port, ms, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    got = bench.max_over_ranks(ms[rank], torch.device("cpu"))
+    agg = bench.aggregate_tflops(world, 1e12, got)
+    q.put((rank, got, agg))
+    torch.distributed.destroy_process_group()
+
+
+def test_bench_takes_max_over_two_gloo_ranks():
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    ms = [2.0, 5.0]
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, ms, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, got, agg in out:
+        assert got == 5.0
+        assert abs(agg - 2 * 1e12 / 5e-3 / 1e12) < 1e-9
