@@ -6,21 +6,32 @@
 // 128 tokens of each kept key block only; tiles that are not kept are never
 // loaded or multiplied.
 //
-// One CTA per (head, query block) row, 256 threads, warp-specialised:
-//   warp 0 lane 0  producer: TMA of the Q tile (straight from token layout:
-//                  a rank-4 box of 2 x 8 x 8 tokens x 64 dims, so the window
-//                  partition costs nothing) and of each kept K/V tile (block
-//                  layout in the ring, two 16 KB boxes per tile) into a
-//                  3-stage shared-memory ring, 128-byte swizzled;
-//   warp 1 lane 0  MMA issuer: S = Q K^T (tcgen05.mma, both operands in
-//                  shared memory, fp32 accumulator in TMEM, double-buffered)
-//                  and O += P V (P read from TMEM, V from shared memory);
-//   warps 4-7      softmax: one query row per thread; reads S from TMEM,
-//                  online softmax in the log2 domain with lazy rescaling of O
-//                  (only when the row maximum grew by more than 2^8), writes
-//                  P as bf16 back over S, and finally normalises O and stores
-//                  it with a TMA store into token layout (reverse partition).
-// TMEM: S0 cols [0,128), S1 [128,256), O [256,384) of a 512-column allocation.
+// Persistent kernel: one CTA per SM walks the (head, query block) rows
+// blockIdx.x, blockIdx.x + gridDim.x, ... (head-major, so the CTAs running at
+// the same time share the key/value tiles of one or two heads in L2).
+// 384 threads, warp-specialised:
+//   warp 0         producer: validates each row's kept list (whole warp), then
+//                  lane 0 issues the TMA copies — the Q tile straight from
+//                  token layout (rank-4 box of 2 x 8 x 8 tokens x 64 dims, so
+//                  the window partition costs nothing) into one of two Q
+//                  buffers, and every kept K and V tile (block layout in the
+//                  ring, two 16 KB boxes per tile) into separate K and V
+//                  rings, 128-byte swizzled.  It runs ahead into the next row.
+//   warps 1, 2     MMA issuers, one per softmax group (issuing a tcgen05.mma
+//                  costs its thread ~90 cycles, so one issuer per group keeps
+//                  the tensor pipe fed): S_w = Q K^T (both operands in shared
+//                  memory, fp32 accumulator in TMEM) and O_w += P_w V (P read from
+//                  TMEM, V from shared memory), in dependency order; the PV of a
+//                  tile starts on the first 64 keys while the softmax still
+//                  writes the second half of P.
+//   warps 4-7, 8-11 two softmax warpgroups.  Warpgroup w takes the kept tiles
+//                  j = w, w+2, ... of a row with its own S and O in TMEM: one
+//                  query row per thread, online softmax in the log2 domain with
+//                  lazy rescaling of O (only when the row maximum grew by more
+//                  than 2^8), P written as bf16 over S.  At the end of a row both
+//                  groups merge (m, l, O) and each writes one 64-dim half of the
+//                  bf16 output straight into token layout (reverse partition).
+// TMEM (512 columns): S_w at 128*w, O_w at 256 + 128*w.
 // Every wait is bounded; on expiry the CTA drains its copies and MMAs, frees
 // TMEM and reports LCSA_ERR_TIMEOUT.
 
@@ -31,91 +42,182 @@
 namespace lcsa {
 namespace {
 
-constexpr int kStages = 3;
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
 constexpr uint32_t kTileBytes = 32768;
 constexpr uint32_t kHalfBytes = 16384;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
+constexpr int kSoftmaxWarp0 = 4;
+// Registers: launched at 168 per thread (384 x 168 = 64,512); the control
+// warpgroup gives registers to the two softmax warpgroups:
+// 128 x 80 + 256 x 208 = 63,488 <= 64,512.
+constexpr uint32_t kRegsControl = 80;
+constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kInfoSlots = 4;  // rows the producer may publish ahead of the consumers
 
 struct __align__(1024) AttnSmem {
-    uint8_t q[kTileBytes];  // Q tile; reused as the bf16 output staging tile
-    uint8_t k[kStages][kTileBytes];
-    uint8_t v[kStages][kTileBytes];
-    uint64_t bar_q;
-    uint64_t bar_kfull[kStages];
-    uint64_t bar_vfull[kStages];
-    uint64_t bar_empty[kStages];
+    uint8_t q[2][kTileBytes];  // Q tiles of two consecutive rows; the (m, l) exchange of a
+                               // row's epilogue lives in its Q buffer once its QKs are done
+    uint8_t k[kKStages][kTileBytes];
+    uint8_t v[kVStages][kTileBytes];
+    uint64_t bar_qfull[2];
+    uint64_t bar_qempty[2];
+    uint64_t bar_kfull[kKStages];
+    uint64_t bar_kempty[kKStages];
+    uint64_t bar_vfull[kVStages];
+    uint64_t bar_vempty[kVStages];
     uint64_t bar_sfull[2];
-    uint64_t bar_pfull[2];
-    uint64_t bar_pvdone;
+    uint64_t bar_pfa[2];  // P columns for keys 0-63 written
+    uint64_t bar_pfb[2];  // P columns for keys 64-127 written (and O rescaled)
+    uint64_t bar_pvdone[2];
     uint64_t bar_ofinal;
-    uint64_t bar_drain;
+    uint64_t bar_ofree;
+    uint64_t bar_drain[2];
+    uint64_t bar_info_full[kInfoSlots];
+    uint64_t bar_info_empty[kInfoSlots];
+    int32_t info_n[kInfoSlots];  // validated kept count of row r in slot r % kInfoSlots
     uint32_t tmem_base;
-    int32_t n_tiles;
     int32_t abort_word;
 };
 
+__device__ __forceinline__ uint32_t col_s(int w) { return static_cast<uint32_t>(w) * 128u; }
+__device__ __forceinline__ uint32_t col_o(int w) { return 256u + static_cast<uint32_t>(w) * 128u; }
+
+// Kept tiles of a row, or 0 when its count or an index is out of range (whole warp).
+__device__ __forceinline__ int row_tiles(const AttnArgs &a, int unit, int lane, bool &bad) {
+    const int cnt = a.kept_cnt[unit];
+    bad = cnt < 0 || cnt > a.topk;
+    if (!bad) {
+        const int32_t *row = a.kept_idx + static_cast<size_t>(unit) * a.topk;
+        for (int i = lane; i < cnt; i += 32) {
+            const int j = row[i];
+            bad |= (j < 0 || j >= a.n_key_blocks);
+        }
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    return bad ? 0 : cnt;
+}
+
+struct RowGeom {
+    int h, ql, qby, qbx, frame0;
+};
+
+__device__ __forceinline__ RowGeom row_geom(const AttnArgs &a, int unit) {
+    RowGeom g;
+    const int nq = a.q_layers * a.nblk;
+    g.h = unit / nq;
+    const int qi = unit - g.h * nq;
+    g.ql = qi / a.nblk;
+    const int qb = qi - g.ql * a.nblk;
+    g.qby = qb / a.grid_w;
+    g.qbx = qb - g.qby * a.grid_w;
+    g.frame0 = g.h * a.tq + g.ql * 2;  // first frame of the block in the Q/O maps
+    return g;
+}
+
+// Descriptors of the first Q / K / V buffer; buffer i starts i * 32 KB later,
+// which only moves the start-address field (addresses stay below 256 KB).
+struct MmaCtx {
+    uint32_t tmem, idesc_qk, idesc_pv;
+    uint64_t qdesc0, kdesc0, vdesc0;
+};
+constexpr uint64_t kTileDescStep = kTileBytes >> 4;
+
+// S_w = Q K_j^T for tile j of the current row (w = j & 1); t = the group's
+// running tile count (all rows), gk = the running tile count of the CTA.
+__device__ __forceinline__ bool issue_qk(AttnSmem &sm, const MmaCtx &m, int qb, int w, int t, int gk,
+                                         volatile int *abort_word, uint64_t to) {
+    const int ks = gk % kKStages;
+    if (!mbar_wait(smem_u32(&sm.bar_kfull[ks]), (gk / kKStages) & 1, abort_word, to)) return false;
+    // S_w also holds P of this group's previous tile: that PV must have finished.
+    if (t >= 1 && !mbar_wait(smem_u32(&sm.bar_pvdone[w]), (t - 1) & 1, abort_word, to)) return false;
+    tc_fence_after();
+    const uint64_t qd = m.qdesc0 + qb * kTileDescStep, kd = m.kdesc0 + ks * kTileDescStep;
+    const uint32_t d = m.tmem + col_s(w);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        // K-major Q and K: 16 dims = 32 bytes per MMA inside the 128-byte
+        // swizzle row; dims 64-127 live in the second 16 KB half.
+        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+        mma_ss(d, qd + off, kd + off, m.idesc_qk, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(smem_u32(&sm.bar_sfull[w]));
+    mma_commit(smem_u32(&sm.bar_kempty[ks]));
+    return true;
+}
+
+// O_w += P_w V_j for the group's tile; `first` = its first tile of the row.
+__device__ __forceinline__ bool issue_pv(AttnSmem &sm, const MmaCtx &m, int w, int t, int gk, bool first, int act,
+                                         volatile int *abort_word, uint64_t to) {
+    const int vs = gk % kVStages;
+    if (!mbar_wait(smem_u32(&sm.bar_vfull[vs]), (gk / kVStages) & 1, abort_word, to)) return false;
+    // The first PV of a row overwrites O_w: the previous row's epilogue must
+    // have read both accumulators.
+    if (first && act >= 1 && !mbar_wait(smem_u32(&sm.bar_ofree), (act - 1) & 1, abort_word, to)) return false;
+    const uint64_t vd = m.vdesc0 + vs * kTileDescStep;
+    const uint32_t d = m.tmem + col_o(w), p = m.tmem + col_s(w);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        // keys 0-63 as soon as their P is written, then keys 64-127
+        const uint32_t bar = smem_u32(half == 0 ? &sm.bar_pfa[w] : &sm.bar_pfb[w]);
+        if (!mbar_wait(bar, t & 1, abort_word, to)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+            // 16 keys per MMA = two 8-row swizzle atoms (2 KB).
+            const int kk = half * 4 + k4;
+            mma_ts(d, p + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4), m.idesc_pv,
+                   (!first || kk > 0) ? 1u : 0u);
+        }
+    }
+    mma_commit(smem_u32(&sm.bar_vempty[vs]));
+    mma_commit(smem_u32(&sm.bar_pvdone[w]));
+    return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                     const AttnArgs a) {
+                     const __grid_constant__ CUtensorMap tm_v, const AttnArgs a, uint16_t *__restrict__ out) {
     extern __shared__ uint8_t smem_raw[];
     AttnSmem &sm = *reinterpret_cast<AttnSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                   ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int unit = blockIdx.x;
-    const int nq = a.q_layers * a.nblk;
-    const int h = unit / nq;
-    const int qi = unit - h * nq;
-    const int ql = qi / a.nblk;
-    const int qb = qi - ql * a.nblk;
-    const int qby = qb / a.grid_w;
-    const int qbx = qb - qby * a.grid_w;
-    const int frame0 = h * a.tq + ql * 2;  // coordinate of the block's first frame in the Q/O maps
     volatile int *abort_word = &sm.abort_word;
     const uint64_t to = a.timeout_ns;
-    const int32_t *kept_row = a.kept_idx + static_cast<size_t>(unit) * a.topk;
 
     if (threadIdx.x == 0) {
-        mbar_init(smem_u32(&sm.bar_q), 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(smem_u32(&sm.bar_kfull[s]), 1);
-            mbar_init(smem_u32(&sm.bar_vfull[s]), 1);
-            mbar_init(smem_u32(&sm.bar_empty[s]), 1);
-        }
         for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&sm.bar_qfull[b]), 1);
+            mbar_init(smem_u32(&sm.bar_qempty[b]), 8);  // one arrival per softmax warp
             mbar_init(smem_u32(&sm.bar_sfull[b]), 1);
-            mbar_init(smem_u32(&sm.bar_pfull[b]), 128);
+            mbar_init(smem_u32(&sm.bar_pfa[b]), 4);     // one arrival per warp of the group
+            mbar_init(smem_u32(&sm.bar_pfb[b]), 4);
+            mbar_init(smem_u32(&sm.bar_drain[b]), 1);
+            mbar_init(smem_u32(&sm.bar_pvdone[b]), 1);
         }
-        mbar_init(smem_u32(&sm.bar_pvdone), 1);
-        mbar_init(smem_u32(&sm.bar_ofinal), 1);
-        mbar_init(smem_u32(&sm.bar_drain), 1);
+        for (int s = 0; s < kKStages; ++s) {
+            mbar_init(smem_u32(&sm.bar_kfull[s]), 1);
+            mbar_init(smem_u32(&sm.bar_kempty[s]), 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            mbar_init(smem_u32(&sm.bar_vfull[s]), 1);
+            mbar_init(smem_u32(&sm.bar_vempty[s]), 1);
+        }
+        mbar_init(smem_u32(&sm.bar_ofinal), 2);  // one commit per MMA issuer
+        mbar_init(smem_u32(&sm.bar_ofree), 8);
+        for (int i = 0; i < kInfoSlots; ++i) {
+            mbar_init(smem_u32(&sm.bar_info_full[i]), 1);
+            mbar_init(smem_u32(&sm.bar_info_empty[i]), 10);  // 2 MMA issuers + 8 softmax warps
+        }
         sm.abort_word = 0;
         fence_mbar_init();
-    }
-    if (warp == 0) {
-        // Validate the kept list of this row before anything is loaded.
-        const int cnt = a.kept_cnt[unit];
-        bool bad = cnt < 0 || cnt > a.topk;
-        if (!bad) {
-            for (int i = lane; i < cnt; i += 32) {
-                const int j = kept_row[i];
-                bad |= (j < 0 || j >= a.n_key_blocks);
-            }
-        }
-        bad = __any_sync(0xffffffffu, bad);
-        if (lane == 0) {
-            sm.n_tiles = bad ? 0 : cnt;
-            if (bad && a.status) atomicOr(a.status, LCSA_ERR_BAD_INDEX);
-            prefetch_tensormap(&tm_q);
-            prefetch_tensormap(&tm_k);
-            prefetch_tensormap(&tm_v);
-            prefetch_tensormap(&tm_o);
-        }
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
@@ -125,226 +227,320 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const int n = sm.n_tiles;
 
-    const uint32_t bar_q = smem_u32(&sm.bar_q);
-    const uint32_t q_smem = smem_u32(sm.q);
-    int issued = 0;  // K/V tiles whose loads the producer issued
+    // Copies issued by the producer (global counters), for the error-path drain.
+    int k_issued = 0, v_issued = 0, q_issued = 0;
 
+    if (warp < kSoftmaxWarp0) setmaxnreg_dec<kRegsControl>();
     if (warp == 0) {
-        if (lane == 0 && n > 0) {
-            // ------------------------------------------------------ producer
-            mbar_arrive_expect_tx(bar_q, kTileBytes);
-            tma_load_4d(q_smem, &tm_q, bar_q, 0, qbx * 8, qby * 8, frame0);
-            tma_load_4d(q_smem + kHalfBytes, &tm_q, bar_q, 64, qbx * 8, qby * 8, frame0);
-            for (int j = 0; j < n; ++j) {
-                const int s = j % kStages;
-                if (j >= kStages &&
-                    !mbar_wait(smem_u32(&sm.bar_empty[s]), ((j / kStages) - 1) & 1, abort_word, to))
-                    break;
-                const int kb = kept_row[j];
-                const int layer = kb / a.nblk;
-                const int b = kb - layer * a.nblk;
-                int slot = a.oldest + layer;
-                if (slot >= a.capacity) slot -= a.capacity;
-                const int r0 = ((slot * a.heads + h) * a.nblk + b) * kBlockTokens;
-                const uint32_t kf = smem_u32(&sm.bar_kfull[s]);
-                const uint32_t vf = smem_u32(&sm.bar_vfull[s]);
-                mbar_arrive_expect_tx(kf, kTileBytes);
-                tma_load_2d(smem_u32(sm.k[s]), &tm_k, kf, 0, r0);
-                tma_load_2d(smem_u32(sm.k[s]) + kHalfBytes, &tm_k, kf, 64, r0);
-                mbar_arrive_expect_tx(vf, kTileBytes);
-                tma_load_2d(smem_u32(sm.v[s]), &tm_v, vf, 0, r0);
-                tma_load_2d(smem_u32(sm.v[s]) + kHalfBytes, &tm_v, vf, 64, r0);
-                issued = j + 1;
-            }
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        if (lane == 0 && n > 0) {
-            // ---------------------------------------------------- MMA issuer
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 1);
-            const uint32_t pvdone = smem_u32(&sm.bar_pvdone);
-            auto issue_pv = [&](int i) -> bool {
-                const int s = i % kStages;
-                const int b = i & 1;
-                if (!mbar_wait(smem_u32(&sm.bar_vfull[s]), (i / kStages) & 1, abort_word, to)) return false;
-                if (!mbar_wait(smem_u32(&sm.bar_pfull[b]), (i >> 1) & 1, abort_word, to)) return false;
-                tc_fence_after();
-                const uint32_t v_smem = smem_u32(sm.v[s]);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    // V is [key][dim]: dims (N) contiguous -> MN-major B operand.
-                    // 16 keys per MMA = two 8-row swizzle atoms (2 KB); the two
-                    // 64-dim halves are 16 KB apart (leading byte offset).
-                    const uint64_t bdesc = smem_desc_sw128(v_smem + kk * 2048, kHalfBytes, 1024);
-                    mma_ts(tmem + kColO, tmem + (b ? 128u : 0u) + kk * 8, bdesc, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        // ---------------------------------------------------------- producer
+        // The whole warp walks the rows: it validates each kept list, publishes
+        // the row's tile count to the consumers, and reads the kept indices 32 at
+        // a time (one coalesced load, then shuffles); lane 0 issues the copies.
+        int g = 0, act = 0, r = 0;  // tiles, non-empty rows and rows so far
+        bool ok = true;
+        for (int unit = blockIdx.x; unit < a.n_units; unit += gridDim.x, ++r) {
+            bool bad;
+            const int n = row_tiles(a, unit, lane, bad);
+            if (lane == 0) {
+                if (bad && a.status) atomicOr(a.status, LCSA_ERR_BAD_INDEX);
+                const int is = r % kInfoSlots;
+                if (r >= kInfoSlots)
+                    ok = mbar_wait(smem_u32(&sm.bar_info_empty[is]), ((r / kInfoSlots) - 1) & 1, abort_word, to);
+                if (ok) {
+                    sm.info_n[is] = n;
+                    mbar_arrive(smem_u32(&sm.bar_info_full[is]));  // release: the count is visible
                 }
-                mma_commit(smem_u32(&sm.bar_empty[s]));
-                mma_commit(pvdone);
-                return true;
-            };
-            bool ok = mbar_wait(bar_q, 0, abort_word, to);
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            if (n == 0) continue;
+            const RowGeom rg = row_geom(a, unit);
+            const int qb = act & 1;
+            if (lane == 0) {
+                if (act >= 2)
+                    ok = mbar_wait(smem_u32(&sm.bar_qempty[qb]), ((act >> 1) - 1) & 1, abort_word, to);
+                if (ok) {
+                    const uint32_t qf = smem_u32(&sm.bar_qfull[qb]);
+                    mbar_arrive_expect_tx(qf, kTileBytes);
+                    tma_load_4d(smem_u32(sm.q[qb]), &tm_q, qf, 0, rg.qbx * 8, rg.qby * 8, rg.frame0);
+                    tma_load_4d(smem_u32(sm.q[qb]) + kHalfBytes, &tm_q, qf, 64, rg.qbx * 8, rg.qby * 8, rg.frame0);
+                    q_issued = act + 1;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            const int32_t *kept_row = a.kept_idx + static_cast<size_t>(unit) * a.topk;
+            int idx = 0;
             for (int j = 0; ok && j < n; ++j) {
-                const int s = j % kStages;
-                const int b = j & 1;
-                if (!mbar_wait(smem_u32(&sm.bar_kfull[s]), (j / kStages) & 1, abort_word, to)) {
-                    ok = false;
-                    break;
+                if ((j & 31) == 0) idx = (j + lane < n) ? __ldg(kept_row + j + lane) : 0;
+                const int kb = __shfl_sync(0xffffffffu, idx, j & 31);
+                if (lane == 0) {
+                    const int gk = g + j;
+                    const int layer = kb / a.nblk;
+                    const int b = kb - layer * a.nblk;
+                    int slot = a.oldest + layer;
+                    if (slot >= a.capacity) slot -= a.capacity;
+                    const int r0 = ((slot * a.heads + rg.h) * a.nblk + b) * kBlockTokens;
+                    const int ks = gk % kKStages;
+                    if (gk >= kKStages)
+                        ok = mbar_wait(smem_u32(&sm.bar_kempty[ks]), ((gk / kKStages) - 1) & 1, abort_word, to);
+                    if (ok) {
+                        const uint32_t kf = smem_u32(&sm.bar_kfull[ks]);
+                        mbar_arrive_expect_tx(kf, kTileBytes);
+                        tma_load_2d(smem_u32(sm.k[ks]), &tm_k, kf, 0, r0);
+                        tma_load_2d(smem_u32(sm.k[ks]) + kHalfBytes, &tm_k, kf, 64, r0);
+                        k_issued = gk + 1;
+                        const int vs = gk % kVStages;
+                        if (gk >= kVStages)
+                            ok = mbar_wait(smem_u32(&sm.bar_vempty[vs]), ((gk / kVStages) - 1) & 1, abort_word, to);
+                        if (ok) {
+                            const uint32_t vf = smem_u32(&sm.bar_vfull[vs]);
+                            mbar_arrive_expect_tx(vf, kTileBytes);
+                            tma_load_2d(smem_u32(sm.v[vs]), &tm_v, vf, 0, r0);
+                            tma_load_2d(smem_u32(sm.v[vs]) + kHalfBytes, &tm_v, vf, 64, r0);
+                            v_issued = gk + 1;
+                        }
+                    }
                 }
-                // S[b] also holds P of tile j-2: wait until that PV finished reading it.
-                if (j >= 2 && !mbar_wait(pvdone, (j - 2) & 1, abort_word, to)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t k_smem = smem_u32(sm.k[s]);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    // K-major Q and K: 16 dims = 32 bytes per MMA inside the
-                    // 128-byte swizzle row; dims 64-127 live in the second half.
-                    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                    mma_ss(tmem + (b ? 128u : 0u), smem_desc_sw128(q_smem + off, 16, 1024),
-                           smem_desc_sw128(k_smem + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(smem_u32(&sm.bar_sfull[b]));
-                if (j >= 1 && !issue_pv(j - 1)) {
-                    ok = false;
-                    break;
-                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             }
-            if (ok) ok = issue_pv(n - 1);
-            if (ok) mma_commit(smem_u32(&sm.bar_ofinal));
-            // Every MMA issued must be complete before TMEM is freed.
-            mma_commit(smem_u32(&sm.bar_drain));
-            mbar_wait_drain(smem_u32(&sm.bar_drain), 0, to);
+            if (!ok) break;
+            g += n;
+            ++act;
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    } else if (warp == 1 || warp == 2) {
+        // ---------------------------------------------- MMA issuer of group w
+        // Tiles j = w, w+2, ... of each row: QK, then per tile PV (as P becomes
+        // available) and the next QK into the same S buffer once that PV completed.
+        const int w = warp - 1;
+        if (lane == 0) {
+            MmaCtx m;
+            m.tmem = tmem;
+            m.idesc_qk = idesc_bf16_f32(128, 128, 0);
+            m.idesc_pv = idesc_bf16_f32(128, 128, 1);
+            // Descriptors of the first buffer of each kind; per-MMA steps only move
+            // the start address.  V is [key][dim]: dims (N) contiguous -> MN-major B
+            // operand, the two 64-dim halves 16 KB apart (leading byte offset).
+            m.qdesc0 = smem_desc_sw128(smem_u32(sm.q[0]), 16, 1024);
+            m.kdesc0 = smem_desc_sw128(smem_u32(sm.k[0]), 16, 1024);
+            m.vdesc0 = smem_desc_sw128(smem_u32(sm.v[0]), kHalfBytes, 1024);
+            int g = 0, act = 0, r = 0;
+            int t = 0;  // tiles of this group so far (all rows)
+            bool ok = true;
+            for (int unit = blockIdx.x; ok && unit < a.n_units; unit += gridDim.x, ++r) {
+                const int is = r % kInfoSlots;
+                if (!(ok = mbar_wait(smem_u32(&sm.bar_info_full[is]), (r / kInfoSlots) & 1, abort_word, to))) break;
+                const int n = *reinterpret_cast<volatile int32_t *>(&sm.info_n[is]);
+                mbar_arrive(smem_u32(&sm.bar_info_empty[is]));
+                if (n == 0) continue;
+                const int qb = act & 1;
+                const int n_mine = (n - w + 1) >> 1;
+                ok = mbar_wait(smem_u32(&sm.bar_qfull[qb]), (act >> 1) & 1, abort_word, to);
+                if (ok && n_mine > 0) ok = issue_qk(sm, m, qb, w, t, g + w, abort_word, to);
+                for (int i = 0; ok && i < n_mine; ++i) {
+                    ok = issue_pv(sm, m, w, t + i, g + w + 2 * i, i == 0, act, abort_word, to);
+                    if (ok && i + 1 < n_mine) ok = issue_qk(sm, m, qb, w, t + i + 1, g + w + 2 * (i + 1), abort_word, to);
+                }
+                if (ok) mma_commit(smem_u32(&sm.bar_ofinal));
+                t += n_mine;
+                g += n;
+                ++act;
+            }
+            // Every MMA issued must be complete before TMEM is freed.
+            mma_commit(smem_u32(&sm.bar_drain[w]));
+            mbar_wait_drain(smem_u32(&sm.bar_drain[w]), 0, to);
+        }
+        __syncwarp();
+    } else if (warp >= kSoftmaxWarp0) {
         // ------------------------------------------------------- softmax
-        const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+        setmaxnreg_inc<kRegsSoftmax>();
+        const int w = (warp - kSoftmaxWarp0) >> 2;  // warpgroup 0 or 1
+        const int quad = warp & 3;                   // TMEM lane quadrant this warp may access
         const int row = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t s_addr = tmem + lane_off + col_s(w);
+        const uint32_t o_addr = tmem + lane_off + col_o(w);
         const float c = a.scale_log2;
-        float m_used = -INFINITY;
-        float l = 0.f;
+        const int tok_t = row >> 6, tok_y = (row >> 3) & 7, tok_x = row & 7;  // token of this row
+        int act = 0, t = 0, r = 0;
         bool ok = true;
-        for (int j = 0; j < n; ++j) {
-            const int b = j & 1;
-            if (j == 0 && (a.flags & LCSA_FLAG_FORCE_TIMEOUT)) {
-                *abort_word = 1;
+        for (int unit = blockIdx.x; unit < a.n_units; unit += gridDim.x, ++r) {
+            const int is = r % kInfoSlots;
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(smem_u32(&sm.bar_info_full[is]), (r / kInfoSlots) & 1, abort_word, to));
+            // both groups leave together when a wait gave up
+            if (!named_bar_and(1, 256, ok)) {
                 ok = false;
                 break;
             }
-            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_sfull[b]), (j >> 1) & 1, abort_word, to));
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t s[128];
-            tmem_ld32(tmem + lane_off + (b ? 128u : 0u) + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-            tmem_ld32(tmem + lane_off + (b ? 128u : 0u) + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-            tmem_ld32(tmem + lane_off + (b ? 128u : 0u) + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-            tmem_ld32(tmem + lane_off + (b ? 128u : 0u) + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-            tmem_wait_ld();
-            float mx = -INFINITY;
+            const int n = *reinterpret_cast<volatile int32_t *>(&sm.info_n[is]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.bar_info_empty[is]));
+            const RowGeom rg = row_geom(a, unit);
+            const size_t tok = (static_cast<size_t>(rg.frame0 + tok_t) * a.tok_h + rg.qby * 8 + tok_y) * a.tok_w +
+                               rg.qbx * 8 + tok_x;
+            uint4 *dst = reinterpret_cast<uint4 *>(out + tok * kHeadDim + w * 64);
+            if (n == 0) {
+                // nothing kept: zeros (lse -inf)
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-            for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
-            const float m_new = mx * c;
-            const bool warp_need = __any_sync(0xffffffffu, m_new > m_used + kRescaleThreshold);
-            float m_next = m_used;
-            float alpha = 1.f;
-            if (warp_need) {
-                m_next = fmaxf(m_used, m_new);
-                alpha = ex2_approx(m_used - m_next);
+                for (int i = 0; i < 8; ++i) dst[i] = z;
+                if (w == 0 && a.lse) a.lse[tok] = -INFINITY;
+                continue;
             }
-            float rs = 0.f;
-            uint32_t pk[64];
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * i]), c, -m_next));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * i + 1]), c, -m_next));
-                rs += p0 + p1;
-                pk[i] = pack_bf16x2(p0, p1);
-            }
-            l = l * alpha + rs;
-            tmem_st32(tmem + lane_off + (b ? 128u : 0u) + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(tmem + lane_off + (b ? 128u : 0u) + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
-            if (warp_need && j > 0) {
-                // O must hold the finished PV of tile j-1 before it is rescaled.
-                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_pvdone), (j - 1) & 1, abort_word, to));
+            const int qb = act & 1;
+            const int n_mine = (n - w + 1) >> 1;  // tiles w, w+2, ...
+            const int n_other = (n - (1 - w) + 1) >> 1;
+            float m_used = -INFINITY;
+            float l = 0.f;
+            for (int i = 0; ok && i < n_mine; ++i, ++t) {
+                if (act == 0 && i == 0 && w == 0 && (a.flags & LCSA_FLAG_FORCE_TIMEOUT)) {
+                    *abort_word = 1;
+                    ok = false;
+                    break;
+                }
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_sfull[w]), t & 1, abort_word, to));
                 if (!ok) break;
                 tc_fence_after();
+                uint32_t s[128];
+                tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+                tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+                tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+                tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+                tmem_wait_ld();
+                // row maximum: eight independent chains, then a small tree
+                float mx8[8];
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t o[32];
-                    tmem_ld32(tmem + lane_off + kColO + cc * 32, o);
-                    tmem_wait_ld();
+                for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(s[e]);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(tmem + lane_off + kColO + cc * 32, o);
+                for (int k = 8; k < 128; k += 8) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], __uint_as_float(s[k + e]));
                 }
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(smem_u32(&sm.bar_pfull[b]));
-            m_used = m_next;
-        }
-        if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_ofinal), 0, abort_word, to));
-        if (ok) {
-            // --------------------------------------------------- epilogue
-            tc_fence_after();
-            const float inv_l = n > 0 ? 1.f / l : 0.f;
-            const uint32_t row_base = q_smem + static_cast<uint32_t>(row) * 128;
+                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                const float m_new = mx * c;
+                const bool warp_need = __any_sync(0xffffffffu, m_new > m_used + kRescaleThreshold);
+                float m_next = m_used;
+                float alpha = 1.f;
+                if (warp_need) {
+                    m_next = fmaxf(m_used, m_new);
+                    alpha = ex2_approx(m_used - m_next);
+                }
+                if (warp_need && i > 0) {
+                    // Rescale O_w before this tile's PV accumulates into it.  O_w is
+                    // stable: the QK of this tile was issued only after the group's
+                    // previous PV completed (it reuses S_w).
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t o[32];
-                if (n > 0) {
-                    tmem_ld32(tmem + lane_off + kColO + cc * 32, o);
-                    tmem_wait_ld();
+                    for (int cc = 0; cc < 4; ++cc) {
+                        uint32_t o[32];
+                        tmem_ld32(o_addr + cc * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                        tmem_st32(o_addr + cc * 32, o);
+                    }
+                }
+                // P = 2^(s*c - m), summed in eight independent chains, packed to bf16
+                // and written over S in two 64-key halves, each announced as soon as
+                // it is in TMEM so that its PV MMAs can start.
+                float sum8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int col = half * 64 + 2 * k;
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(s[col]), c, -m_next));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(s[col + 1]), c, -m_next));
+                        sum8[(2 * k) & 7] += p0;
+                        sum8[(2 * k + 1) & 7] += p1;
+                        pk[k] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st32(s_addr + half * 32, pk);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(half == 0 ? &sm.bar_pfa[w] : &sm.bar_pfb[w]));
+                }
+                const float rs =
+                    ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+                l = l * alpha + rs;
+                m_used = m_next;
+            }
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_ofinal), act & 1, abort_word, to));
+            // both groups take the same decision on going through the epilogue
+            if (!named_bar_and(1, 256, ok && !*abort_word)) {
+                ok = false;
+                break;
+            }
+            // ------------------------------------------------------ epilogue
+            tc_fence_after();
+            float *mlx = reinterpret_cast<float *>(sm.q[qb]);  // every QK of this row completed
+            mlx[(w * 128 + row) * 2 + 0] = m_used;
+            mlx[(w * 128 + row) * 2 + 1] = l;
+            named_bar_sync(2, 256);
+            const float m_o = mlx[((1 - w) * 128 + row) * 2 + 0];
+            const float l_o = mlx[((1 - w) * 128 + row) * 2 + 1];
+            const float m = fmaxf(m_used, m_o);
+            const float a_self = n_mine > 0 ? ex2_approx(m_used - m) : 0.f;
+            const float a_oth = n_other > 0 ? ex2_approx(m_o - m) : 0.f;
+            const float L = l * a_self + l_o * a_oth;
+            const float inv_l = L > 0.f ? 1.f / L : 0.f;
+            const float f_self = a_self * inv_l, f_oth = a_oth * inv_l;
+            // this group writes output dims [64w, 64w+64) of its row
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const uint32_t col = static_cast<uint32_t>(w * 64 + cc * 32);
+                uint32_t o0[32], o1[32];
+                if (n_mine > 0) {
+                    tmem_ld32(tmem + lane_off + col_o(w) + col, o0);
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = 0u;
+                    for (int k = 0; k < 32; ++k) o0[k] = 0u;
                 }
+                if (n_other > 0) {
+                    tmem_ld32(tmem + lane_off + col_o(1 - w) + col, o1);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) o1[k] = 0u;
+                }
+                tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-                // 32 columns = 64 bytes = four 16-byte chunks of the 128-byte
-                // swizzled row of half (cc >> 1); chunk index XOR (row % 8).
-#pragma unroll
-                for (int qd = 0; qd < 4; ++qd) {
-                    const uint32_t chunk = static_cast<uint32_t>((cc & 1) * 4 + qd);
-                    const uint32_t addr = row_base + (cc >> 1) * kHalfBytes + ((chunk ^ (row & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * qd]),
-                                 "r"(pk[4 * qd + 1]), "r"(pk[4 * qd + 2]), "r"(pk[4 * qd + 3])
-                                 : "memory");
+                for (int k = 0; k < 16; ++k) {
+                    const float x0 = __uint_as_float(o0[2 * k]) * f_self + __uint_as_float(o1[2 * k]) * f_oth;
+                    const float x1 = __uint_as_float(o0[2 * k + 1]) * f_self + __uint_as_float(o1[2 * k + 1]) * f_oth;
+                    pk[k] = pack_bf16x2(x0, x1);
                 }
+#pragma unroll
+                for (int qd = 0; qd < 4; ++qd)
+                    dst[cc * 4 + qd] = make_uint4(pk[4 * qd], pk[4 * qd + 1], pk[4 * qd + 2], pk[4 * qd + 3]);
             }
-            if (a.lse) {
-                const int t = row >> 6, y = (row >> 3) & 7, x = row & 7;
-                const size_t idx = (static_cast<size_t>(frame0 + t) * a.tok_h + qby * 8 + y) * a.tok_w + qbx * 8 + x;
-                a.lse[idx] = n > 0 ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
+            if (w == 0 && a.lse) a.lse[tok] = L > 0.f ? (m + __log2f(L)) * kLn2 : -INFINITY;
+            // O of both groups and this Q buffer (the exchange) are free again
+            tc_fence_before();
+            named_bar_sync(3, 256);
+            if (lane == 0) {
+                mbar_arrive(smem_u32(&sm.bar_ofree));
+                mbar_arrive(smem_u32(&sm.bar_qempty[qb]));
             }
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (row == 0) {
-                tma_store_4d(&tm_o, q_smem, 0, qbx * 8, qby * 8, frame0);
-                tma_store_4d(&tm_o, q_smem + kHalfBytes, 64, qbx * 8, qby * 8, frame0);
-                bulk_commit_group();
-                bulk_wait_group_read0();
-            }
+            ++act;
         }
     }
 
     __syncthreads();
-    if (sm.abort_word && warp == 0 && lane == 0 && n > 0) {
+    if (sm.abort_word && warp == 0 && lane == 0) {
         // Error path: every copy still in flight must land before the CTA exits.
-        mbar_wait_drain(bar_q, 0, to);
-        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
-            const int s = j % kStages;
-            mbar_wait_drain(smem_u32(&sm.bar_kfull[s]), (j / kStages) & 1, to);
-            mbar_wait_drain(smem_u32(&sm.bar_vfull[s]), (j / kStages) & 1, to);
-        }
+        for (int i = (q_issued > 2 ? q_issued - 2 : 0); i < q_issued; ++i)
+            mbar_wait_drain(smem_u32(&sm.bar_qfull[i & 1]), (i >> 1) & 1, to);
+        for (int j = (k_issued > kKStages ? k_issued - kKStages : 0); j < k_issued; ++j)
+            mbar_wait_drain(smem_u32(&sm.bar_kfull[j % kKStages]), (j / kKStages) & 1, to);
+        for (int j = (v_issued > kVStages ? v_issued - kVStages : 0); j < v_issued; ++j)
+            mbar_wait_drain(smem_u32(&sm.bar_vfull[j % kVStages]), (j / kVStages) & 1, to);
     }
     if (warp == 1) {
         tc_fence_after();
@@ -356,12 +552,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                             const CUtensorMap &tm_o, const AttnArgs &a, cudaStream_t stream) {
+                             const AttnArgs &a, void *out, cudaStream_t stream) {
     const size_t smem = sizeof(AttnSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    attention_kernel<<<a.n_units, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, tm_o, a);
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const int grid = a.n_units < sms ? a.n_units : sms;
+    attention_kernel<<<grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, a, static_cast<uint16_t *>(out));
     return cudaGetLastError();
 }
 

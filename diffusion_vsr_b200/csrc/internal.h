@@ -31,7 +31,7 @@ struct AttnArgs {
 };
 
 cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                             const CUtensorMap &tm_o, const AttnArgs &a, cudaStream_t stream);
+                             const AttnArgs &a, void *out, cudaStream_t stream);
 
 // Draft mask: q block means, scores over allowed candidates, top-k.
 struct DraftArgs {
@@ -40,6 +40,7 @@ struct DraftArgs {
     int32_t heads, grid_h, grid_w, nblk, q_layers, tq, tok_h, tok_w;
     int32_t capacity, oldest, count;
     int32_t local_range, local_mode, topk;
+    int32_t cand_cap;      // allowed candidates of the widest row, rounded up to 32
     float scale;
     int32_t *kept_idx;
     int32_t *kept_cnt;

@@ -184,7 +184,8 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
     if (rc != LCSA_OK) return rc;
     if ((rc = check_params(p, cache)) != LCSA_OK) return rc;
     if (!q_tok || !aligned16(q_tok) || !kept_idx || !kept_cnt) return LCSA_ERR_INVALID_ARG;
-    if (max_candidates(p, cache) > lcsa::kMaxCandidates) return LCSA_ERR_INVALID_ARG;
+    const int64_t cand = max_candidates(p, cache);
+    if (cand > lcsa::kMaxCandidates) return LCSA_ERR_INVALID_ARG;
     if ((rc = check_device()) != LCSA_OK) return rc;
 
     lcsa::DraftArgs a{};
@@ -204,6 +205,7 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
     a.local_range = p->local_range;
     a.local_mode = p->local_mode;
     a.topk = p->topk;
+    a.cand_cap = static_cast<int32_t>((cand + 31) / 32 * 32);
     a.scale = eff_scale(p);
     a.kept_idx = kept_idx;
     a.kept_cnt = kept_cnt;
@@ -227,9 +229,8 @@ int lcsa_attention(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache 
     const int nblk = p->grid_h * p->grid_w;
     const int64_t frames = static_cast<int64_t>(p->heads) * 2 * p->q_layers;
     const int64_t rows = static_cast<int64_t>(cache->capacity) * cache->heads * nblk * kBlockTokens;
-    CUtensorMap tq, tk, tv, to;
-    if (!make_token_map(&tq, q_tok, frames, 8 * p->grid_h, 8 * p->grid_w) ||
-        !make_token_map(&to, out_tok, frames, 8 * p->grid_h, 8 * p->grid_w) || !make_ring_map(&tk, cache->k, rows) ||
+    CUtensorMap tq, tk, tv;
+    if (!make_token_map(&tq, q_tok, frames, 8 * p->grid_h, 8 * p->grid_w) || !make_ring_map(&tk, cache->k, rows) ||
         !make_ring_map(&tv, cache->v, rows))
         return LCSA_ERR_CUDA;
 
@@ -254,7 +255,7 @@ int lcsa_attention(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache 
     a.status = d_status;
     a.timeout_ns = lcsa::kWatchdogNs;
     a.flags = p->flags;
-    if (lcsa::launch_attention(tq, tk, tv, to, a, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (lcsa::launch_attention(tq, tk, tv, a, out_tok, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LCSA_ERR_CUDA;
     return LCSA_OK;
 }
