@@ -128,12 +128,16 @@ constexpr uint64_t kTileDescStep = kTileBytes >> 4;
 
 // S_w = Q K_j^T for tile j of the current row (w = j & 1); t = the group's
 // running tile count (all rows), gk = the running tile count of the CTA.
-__device__ __forceinline__ bool issue_qk(AttnSmem &sm, const MmaCtx &m, int qb, int w, int t, int gk,
+// prev_t >= 0: the CTA's previous tile belongs to the other group as its tile
+// prev_t; this QK starts only once that QK completed, so the two groups' QKs
+// alternate on the tensor pipe and their softmaxes run staggered.
+__device__ __forceinline__ bool issue_qk(AttnSmem &sm, const MmaCtx &m, int qb, int w, int t, int gk, int prev_t,
                                          volatile int *abort_word, uint64_t to) {
     const int ks = gk % kKStages;
     if (!mbar_wait(smem_u32(&sm.bar_kfull[ks]), (gk / kKStages) & 1, abort_word, to)) return false;
     // S_w also holds P of this group's previous tile: that PV must have finished.
     if (t >= 1 && !mbar_wait(smem_u32(&sm.bar_pvdone[w]), (t - 1) & 1, abort_word, to)) return false;
+    if (prev_t >= 0 && !mbar_wait(smem_u32(&sm.bar_sfull[1 - w]), prev_t & 1, abort_word, to)) return false;
     tc_fence_after();
     const uint64_t qd = m.qdesc0 + qb * kTileDescStep, kd = m.kdesc0 + ks * kTileDescStep;
     const uint32_t d = m.tmem + col_s(w);
@@ -326,7 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             m.kdesc0 = smem_desc_sw128(smem_u32(sm.k[0]), 16, 1024);
             m.vdesc0 = smem_desc_sw128(smem_u32(sm.v[0]), kHalfBytes, 1024);
             int g = 0, act = 0, r = 0;
-            int t = 0;  // tiles of this group so far (all rows)
+            int t = 0;      // tiles of this group so far (all rows)
+            int t_oth = 0;  // tiles of the other group before the current row
+            int n_prev = 0; // tiles of the previous non-empty row
             bool ok = true;
             for (int unit = blockIdx.x; ok && unit < a.n_units; unit += gridDim.x, ++r) {
                 const int is = r % kInfoSlots;
@@ -337,13 +343,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int qb = act & 1;
                 const int n_mine = (n - w + 1) >> 1;
                 ok = mbar_wait(smem_u32(&sm.bar_qfull[qb]), (act >> 1) & 1, abort_word, to);
-                if (ok && n_mine > 0) ok = issue_qk(sm, m, qb, w, t, g + w, abort_word, to);
+                // Tile w + 2i of the row follows tile w + 2i - 1 of the other group
+                // (for group 0's first tile: the previous row's last tile, when
+                // that row had an even count).
+                auto prev_of = [&](int i) -> int {
+                    if (w == 1) return t_oth + i;
+                    if (i >= 1) return t_oth + i - 1;
+                    return (act >= 1 && (n_prev & 1) == 0) ? t_oth - 1 : -1;
+                };
+                if (ok && n_mine > 0) ok = issue_qk(sm, m, qb, w, t, g + w, prev_of(0), abort_word, to);
                 for (int i = 0; ok && i < n_mine; ++i) {
                     ok = issue_pv(sm, m, w, t + i, g + w + 2 * i, i == 0, act, abort_word, to);
-                    if (ok && i + 1 < n_mine) ok = issue_qk(sm, m, qb, w, t + i + 1, g + w + 2 * (i + 1), abort_word, to);
+                    if (ok && i + 1 < n_mine)
+                        ok = issue_qk(sm, m, qb, w, t + i + 1, g + w + 2 * (i + 1), prev_of(i + 1), abort_word, to);
                 }
+                // An issuer without a tile in this row has not waited for the
+                // previous row's epilogue (its first PV would have): wait here,
+                // so that its commit cannot count toward the previous row's
+                // phase of bar_ofinal.
+                if (ok && n_mine == 0 && act >= 1)
+                    ok = mbar_wait(smem_u32(&sm.bar_ofree), (act - 1) & 1, abort_word, to);
                 if (ok) mma_commit(smem_u32(&sm.bar_ofinal));
                 t += n_mine;
+                t_oth += n - n_mine;
+                n_prev = n;
                 g += n;
                 ++act;
             }

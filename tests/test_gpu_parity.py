@@ -127,24 +127,29 @@ def test_deterministic_byte_identical():
 
 # ------------------------------------------------------------------ edge cases
 
-def _tiny_setup(topk=8):
+def _tiny_setup(topk=8, heads=None):
+    import dataclasses
     L = _lib()
     w = W.WORKLOADS["tiny"]
+    if heads is not None:
+        w = dataclasses.replace(w, heads=heads)
     q, k, v = [t.cuda() for t in W.gen_layers(w, 0, w.q_layers)]
     layer = L.LcsaLayer(w.heads, w.grid_h, w.grid_w, w.q_layers, w.kv_len, topk, device="cuda")
     layer.append(k, v)
     return L, w, q, k, v, layer
 
 
-def test_zero_and_single_tile_rows():
-    L, w, q, k, v, layer = _tiny_setup(topk=4)
+def _check_ragged_rows(heads, counts, seed):
+    """Attention over hand-made kept lists with `counts` tiles per row."""
+    topk = 4
+    L, w, q, k, v, layer = _tiny_setup(topk=topk, heads=heads)
     Nq = w.n_query_blocks
-    kept = torch.full((w.heads, Nq, 4), -1, dtype=torch.int32)
+    kept = torch.full((w.heads, Nq, topk), -1, dtype=torch.int32)
     cnt = torch.zeros((w.heads, Nq), dtype=torch.int32)
-    rng = np.random.default_rng(3)
+    rng = np.random.default_rng(seed)
     for h in range(w.heads):
         for i in range(Nq):
-            c = int(rng.integers(0, 5))  # 0..4 tiles, ragged
+            c = int(rng.choice(counts))
             sel = np.sort(rng.choice(32, size=c, replace=False))
             kept[h, i, :c] = torch.from_numpy(sel.astype(np.int32))
             cnt[h, i] = c
@@ -152,7 +157,7 @@ def test_zero_and_single_tile_rows():
     lse = torch.empty(q.shape[:4], dtype=torch.float32, device="cuda")
     L.lcsa_attention(layer.params, q, layer.cache, kept.cuda(), cnt.cuda(), out, lse, d_status=layer.status)
     torch.cuda.synchronize()
-    assert layer.status.item() == 0
+    assert layer.status.item() == 0, L.status_string(layer.status.item())
     qb = O.partition(Hn.f32(q))
     kb = O.partition(Hn.f32(k))
     vb = O.partition(Hn.f32(v))
@@ -166,6 +171,18 @@ def test_zero_and_single_tile_rows():
             else:
                 assert np.max(np.abs(ob[h, i] - ro)) <= Hn.ATOL_OUT
                 assert np.max(np.abs(lb[h, i] - rl)) <= 2e-3
+
+
+def test_zero_and_single_tile_rows():
+    # 64 rows: one row per CTA, 0..4 tiles each
+    _check_ragged_rows(heads=None, counts=[0, 1, 2, 3, 4], seed=3)
+
+
+def test_consecutive_single_tile_rows_in_one_cta():
+    # 12 heads x 32 query blocks = 384 rows over at most 148 persistent CTAs:
+    # every CTA walks two or three rows, mostly with a single kept tile, so the
+    # second MMA issuer often has no tile in two rows in a row.
+    _check_ragged_rows(heads=12, counts=[0, 1, 1, 1, 1, 2], seed=5)
 
 
 def test_bad_kept_index_is_reported_and_row_zeroed():
