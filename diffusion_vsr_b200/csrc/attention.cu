@@ -22,8 +22,10 @@
 //                  the tensor pipe fed): S_w = Q K^T (both operands in shared
 //                  memory, fp32 accumulator in TMEM) and O_w += P_w V (P read from
 //                  TMEM, V from shared memory), in dependency order; the PV of a
-//                  tile starts on the first 64 keys while the softmax still
-//                  writes the second half of P.
+//                  tile runs quarter by quarter (32 keys) as the softmax writes
+//                  P.  A QK starts only once the CTA's previous QK (the other
+//                  group's) completed, so the two groups run staggered: one
+//                  group's softmax overlaps the other group's MMAs.
 //   warps 4-7, 8-11 two softmax warpgroups.  Warpgroup w takes the kept tiles
 //                  j = w, w+2, ... of a row with its own S and O in TMEM: one
 //                  query row per thread, online softmax in the log2 domain with
@@ -70,8 +72,8 @@ struct __align__(1024) AttnSmem {
     uint64_t bar_vfull[kVStages];
     uint64_t bar_vempty[kVStages];
     uint64_t bar_sfull[2];
-    uint64_t bar_pfa[2];  // P columns for keys 0-63 written
-    uint64_t bar_pfb[2];  // P columns for keys 64-127 written (and O rescaled)
+    uint64_t bar_pq[4][2];  // [quarter][group]: P of keys 32q..32q+31 written (quarter 0:
+                            // also O rescaled)
     uint64_t bar_pvdone[2];
     uint64_t bar_ofinal;
     uint64_t bar_ofree;
@@ -124,6 +126,7 @@ struct MmaCtx {
     uint32_t tmem, idesc_qk, idesc_pv;
     uint64_t qdesc0, kdesc0, vdesc0;
 };
+
 constexpr uint64_t kTileDescStep = kTileBytes >> 4;
 
 // S_w = Q K_j^T for tile j of the current row (w = j & 1); t = the group's
@@ -164,15 +167,15 @@ __device__ __forceinline__ bool issue_pv(AttnSmem &sm, const MmaCtx &m, int w, i
     const uint64_t vd = m.vdesc0 + vs * kTileDescStep;
     const uint32_t d = m.tmem + col_o(w), p = m.tmem + col_s(w);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        // keys 0-63 as soon as their P is written, then keys 64-127
-        const uint32_t bar = smem_u32(half == 0 ? &sm.bar_pfa[w] : &sm.bar_pfb[w]);
+    for (int qq = 0; qq < 4; ++qq) {
+        // each quarter of 32 keys as soon as its P is written
+        const uint32_t bar = smem_u32(&sm.bar_pq[qq][w]);
         if (!mbar_wait(bar, t & 1, abort_word, to)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
+        for (int k4 = 0; k4 < 2; ++k4) {
             // 16 keys per MMA = two 8-row swizzle atoms (2 KB).
-            const int kk = half * 4 + k4;
+            const int kk = qq * 2 + k4;
             mma_ts(d, p + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4), m.idesc_pv,
                    (!first || kk > 0) ? 1u : 0u);
         }
@@ -198,8 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&sm.bar_qfull[b]), 1);
             mbar_init(smem_u32(&sm.bar_qempty[b]), 8);  // one arrival per softmax warp
             mbar_init(smem_u32(&sm.bar_sfull[b]), 1);
-            mbar_init(smem_u32(&sm.bar_pfa[b]), 4);     // one arrival per warp of the group
-            mbar_init(smem_u32(&sm.bar_pfb[b]), 4);
+            for (int qq = 0; qq < 4; ++qq) mbar_init(smem_u32(&sm.bar_pq[qq][b]), 4);  // one arrival per warp
             mbar_init(smem_u32(&sm.bar_drain[b]), 1);
             mbar_init(smem_u32(&sm.bar_pvdone[b]), 1);
         }
@@ -466,28 +468,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 // P = 2^(s*c - m), summed in eight independent chains, packed to bf16
-                // and written over S in two 64-key halves, each announced as soon as
-                // it is in TMEM so that its PV MMAs can start.
+                // and written over S in four 32-key quarters, each announced as soon
+                // as it is in TMEM so that its PV MMAs can start.
                 float sum8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t pk[32];
+                for (int qq = 0; qq < 4; ++qq) {
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const int col = half * 64 + 2 * k;
+                    for (int k = 0; k < 16; ++k) {
+                        const int col = qq * 32 + 2 * k;
                         const float p0 = ex2_approx(fmaf(__uint_as_float(s[col]), c, -m_next));
                         const float p1 = ex2_approx(fmaf(__uint_as_float(s[col + 1]), c, -m_next));
                         sum8[(2 * k) & 7] += p0;
                         sum8[(2 * k + 1) & 7] += p1;
                         pk[k] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st32(s_addr + half * 32, pk);
+                    tmem_st16(s_addr + qq * 16, pk);
                     tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(half == 0 ? &sm.bar_pfa[w] : &sm.bar_pfb[w]));
+                    if (lane == 0) mbar_arrive(smem_u32(&sm.bar_pq[qq][w]));
                 }
                 const float rs =
                     ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));

@@ -9,22 +9,22 @@
 // softmax of the page is monotone and does not change the selection, so it
 // is not computed.
 //
-// One CTA (8 warps) per group of 8 consecutive query blocks of one head and
-// block-layer.  Neighbouring query blocks have overlapping windows, so the
-// key-block means are read once per group:
-//  1. warp w computes the mean of query block w: lane l owns dims
-//     [4l, 4l+4), one coalesced 256-byte token row per load, 32 loads in
-//     flight, fp32 sums in token order, times 1/128 (deterministic);
-//  2. one candidate of the union of the 8 windows per thread, enumerated in
-//     ascending key index: its 512-byte mean is loaded once and dotted (fp32)
-//     with every query mean of the group whose own window contains it;
-//     candidates outside a block's window get a sentinel key;
-//  3. warp w selects for query block w the k = min(topk, allowed) best
-//     exactly: scores become 32-bit keys whose unsigned order is descending
-//     score; a 4-pass radix select (8 bits per pass, warp histogram in shared
-//     memory) finds the k-th key T; the kept set is every key < T plus the
-//     first (lowest-index) keys equal to T, written in ascending key index by
-//     a ballot compaction.
+// One CTA of 8 warps per (head, query block) row, so that every SM holds
+// several rows at once and each phase is a single round trip to memory:
+//  1. block mean of q: warp w sums tokens [16w, 16w + 16) of the block
+//     (16-byte loads, a half-warp per token, 8 tokens in flight per lane),
+//     the 8 partial sums are added in a fixed tree order, times 1/128
+//     (deterministic);
+//  2. the allowed candidates, enumerated in ascending key index (layer, then
+//     window row, then window column), eight per warp at a time: each 512-byte
+//     key mean is one coalesced warp load, dotted with the q mean in fp32
+//     (per-lane partial products, then a fixed reduce-scatter butterfly);
+//  3. exact top-k: scores become 32-bit keys whose unsigned order is the
+//     descending score order; a 4-pass radix select (8 bits per pass, block
+//     histogram in shared memory, one atomic per distinct bin and warp) finds
+//     the k-th key T; warp 0 writes every
+//     key < T plus the first (lowest-index) keys equal to T, in ascending key
+//     index, by a ballot compaction.
 
 #include <cfloat>
 
@@ -35,10 +35,9 @@
 namespace lcsa {
 namespace {
 
-constexpr int kG = 8;  // query blocks per CTA (one warp each)
-constexpr int kThreads = kG * 32;
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
 constexpr uint32_t kFull = 0xffffffffu;
-constexpr uint32_t kNotCandidate = 0xFFFFFFFFu;
 
 __device__ __forceinline__ void window_1d(int i, int n, int r, int mode, int &lo, int &hi) {
     // Allowed block range [lo, hi) along one axis of the block grid.
@@ -58,13 +57,19 @@ __device__ __forceinline__ void window_1d(int i, int n, int r, int mode, int &lo
 }
 
 // 32-bit key whose unsigned ascending order is the descending order of the
-// score (-0 is folded onto +0 so that the two tie).  Finite scores never map
-// to the sentinel 0xFFFFFFFF.
+// score (-0 is folded onto +0 so that the two tie).
 __device__ __forceinline__ uint32_t desc_key(float score) {
     uint32_t u = __float_as_uint(score);
     if (u == 0x80000000u) u = 0u;
     const uint32_t ordered = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
     return ~ordered;
+}
+
+// Exact n / d for 0 <= n, d < 2^16 (d >= 1) with m = ceil(2^32 / d): the
+// rounding excess of n m / 2^32 over n / d is below n / 2^32 < 1 / d.
+__device__ __forceinline__ uint64_t div_magic(uint32_t d) { return ((1ull << 32) + d - 1) / d; }
+__device__ __forceinline__ int div_by(int n, uint64_t m) {
+    return static_cast<int>((static_cast<uint64_t>(static_cast<uint32_t>(n)) * m) >> 32);
 }
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
@@ -74,222 +79,228 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 }
 
 struct DraftSmem {
-    __align__(16) float mq[kG][kHeadDim];
-    uint32_t hist[kG][256];
-    int win[kG][4];  // y0, y1, x0, x1 of each block's window; y0 = -1 for no block
+    __align__(16) float part[kWarps][kHeadDim];  // per-warp partial sums of q
+    __align__(16) float mq[kHeadDim];
+    uint32_t hist[256];
+    uint32_t digit, below;
 };
 
-// Exact k-th smallest of the candidate keys in keys[0, n) (sentinels skipped,
-// 1 <= k <= candidates): returns its value; k_eq = how many keys equal to it
-// belong to the k smallest.  Whole warp.
-__device__ uint32_t radix_select(const uint32_t *keys, int n, int k, uint32_t *hist, int lane, int &k_eq) {
-    uint32_t prefix = 0, mask = 0;
-    uint32_t k_rem = static_cast<uint32_t>(k);
+__global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
+    __shared__ DraftSmem sm;
+    extern __shared__ uint32_t keys[];  // [cand_cap]
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int unit = blockIdx.x;  // (head, query layer, query block) row
+    const int qb = unit % a.nblk;
+    const int ql = (unit / a.nblk) % a.q_layers;
+    const int h = unit / (a.nblk * a.q_layers);
+    const int qby = qb / a.grid_w;
+    const int qbx = qb - qby * a.grid_w;
+
+    // ---- 1. block mean of q
+    {
+        const size_t frame = static_cast<size_t>(h) * a.tq + ql * 2;
+        const int half = lane >> 4, d8 = lane & 15;  // token parity, dims [8 d8, 8 d8 + 8)
+        uint4 raw[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {  // tokens n = 16 w + 2 i + half, (t, y, x) row-major
+            const int n = warp * 16 + 2 * i + half;
+            const int t = n >> 6, y = (n >> 3) & 7, x = n & 7;
+            const size_t tok = ((frame + t) * a.tok_h + qby * 8 + y) * a.tok_w + qbx * 8 + x;
+            raw[i] = __ldg(reinterpret_cast<const uint4 *>(a.q + tok * kHeadDim) + d8);
+        }
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t w4[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc[2 * e] += __uint_as_float(w4[e] << 16);
+                acc[2 * e + 1] += __uint_as_float(w4[e] & 0xFFFF0000u);
+            }
+        }
+        // even tokens (lanes 0-15) + odd tokens (lanes 16-31)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float o = __shfl_xor_sync(kFull, acc[e], 16);
+            acc[e] = half == 0 ? acc[e] + o : o + acc[e];
+        }
+        if (half == 0) {
+            float4 *dst = reinterpret_cast<float4 *>(&sm.part[warp][8 * d8]);
+            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
+    }
+    int y0, y1, x0, x1;
+    window_1d(qby, a.grid_h, a.local_range, a.local_mode, y0, y1);
+    window_1d(qbx, a.grid_w, a.local_range, a.local_mode, x0, x1);
+    const int wx = x1 - x0;
+    const int wsz = (y1 - y0) * wx;
+    const int n_layers = a.count - a.q_layers + ql + 1;  // key layers up to this block's own
+    const int ncand = n_layers * wsz;                   // >= 1 (the block itself)
+    const uint64_t m_wsz = div_magic(static_cast<uint32_t>(wsz)), m_wx = div_magic(static_cast<uint32_t>(wx));
+    const int n_keys = a.count * a.nblk;
+    float *srow = a.scores ? a.scores + static_cast<size_t>(unit) * n_keys : nullptr;
+    if (srow) {
+        for (int j = tid; j < n_keys; j += kThreads) srow[j] = -INFINITY;
+    }
+    __syncthreads();
+    if (tid < kHeadDim) {
+        const float (*p)[kHeadDim] = sm.part;
+        const float s = ((p[0][tid] + p[1][tid]) + (p[2][tid] + p[3][tid])) +
+                        ((p[4][tid] + p[5][tid]) + (p[6][tid] + p[7][tid]));
+        const float m = s * (1.0f / 128.0f);
+        sm.mq[tid] = m;
+        if (a.qmean) a.qmean[static_cast<size_t>(unit) * kHeadDim + tid] = m;
+    }
+    __syncthreads();  // q mean and the -inf prefill are visible to every thread
+
+    // ---- 2. scores of the allowed candidates: warp w takes candidates
+    //         64i + 8w ... 64i + 8w + 7; lane l reads dims [4l, 4l + 4) of each
+    //         (one coalesced 512-byte row per load, 8 in flight), fp32
+    //         products, then a fixed reduce-scatter butterfly.
+    {
+        constexpr int kU = 8;
+        const float4 qv = reinterpret_cast<const float4 *>(sm.mq)[lane];
+        for (int c0 = warp * kU; c0 < ncand; c0 += kWarps * kU) {
+            // lane u < kU locates candidate c0 + u (one division pair per lane),
+            // then every lane loads its 16 bytes of each of the kU rows
+            const float4 *row = nullptr;
+            int jl = 0;
+            if (lane < kU) {
+                const int c = min(c0 + lane, ncand - 1);
+                const int layer = div_by(c, m_wsz);
+                const int rem = c - layer * wsz;
+                const int ry = div_by(rem, m_wx);
+                const int yy = y0 + ry;
+                const int xx = x0 + rem - ry * wx;
+                const int b = yy * a.grid_w + xx;
+                int slot = a.oldest + layer;
+                if (slot >= a.capacity) slot -= a.capacity;
+                jl = layer * a.nblk + b;
+                row = reinterpret_cast<const float4 *>(a.kmean + ((static_cast<size_t>(slot) * a.heads + h) * a.nblk + b) *
+                                                                     kHeadDim);
+            }
+            float4 kv[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const float4 *ru = reinterpret_cast<const float4 *>(
+                    __shfl_sync(kFull, reinterpret_cast<unsigned long long>(row), u));
+                kv[u] = __ldg(ru + lane);
+            }
+            float dot[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                float d = qv.x * kv[u].x;
+                d = fmaf(qv.y, kv[u].y, d);
+                d = fmaf(qv.z, kv[u].z, d);
+                dot[u] = fmaf(qv.w, kv[u].w, d);
+            }
+            // reduce-scatter over the lanes: after the xor-16, -8 and -4 steps
+            // lane l holds candidate 4 b4 + 2 b3 + b2 (b = bits of l) summed over
+            // 8 lanes; xor-2 and xor-1 complete the 32-lane sum
+            const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+            float d4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float keep = b4 ? dot[i + 4] : dot[i];
+                const float send = b4 ? dot[i] : dot[i + 4];
+                d4[i] = keep + __shfl_xor_sync(kFull, send, 16);
+            }
+            float d2[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float keep = b3 ? d4[i + 2] : d4[i];
+                const float send = b3 ? d4[i] : d4[i + 2];
+                d2[i] = keep + __shfl_xor_sync(kFull, send, 8);
+            }
+            float d1 = (b2 ? d2[1] : d2[0]) + __shfl_xor_sync(kFull, b2 ? d2[0] : d2[1], 4);
+            d1 += __shfl_xor_sync(kFull, d1, 2);
+            d1 += __shfl_xor_sync(kFull, d1, 1);
+            const int u = lane >> 2;
+            const int jl_u = __shfl_sync(kFull, jl, u);
+            if ((lane & 3) == 0 && c0 + u < ncand) {
+                const float score = d1 * a.scale;
+                keys[c0 + u] = desc_key(score);
+                if (srow) srow[jl_u] = score;
+            }
+        }
+    }
+
+    // ---- 3. exact top-k: radix select of the k-th smallest key
+    const int k = min(a.topk, ncand);
+    uint32_t prefix = 0, mask = 0, k_rem = static_cast<uint32_t>(k);
 #pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
-        for (int b = lane; b < 256; b += 32) hist[b] = 0u;
-        __syncwarp();
-        for (int c = lane; c < n; c += 32) {
-            const uint32_t key = keys[c];
-            if (key != kNotCandidate && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        sm.hist[tid] = 0u;  // kThreads == 256 bins
+        __syncthreads();    // (first pass: also the keys of phase 2)
+        for (int c0 = warp * 32; c0 < ncand; c0 += kThreads) {  // whole warps, one add per distinct bin
+            const int c = c0 + lane;
+            const uint32_t key = c < ncand ? keys[c] : 0u;
+            const bool hit = c < ncand && (key & mask) == prefix;
+            const uint32_t bin = hit ? ((key >> shift) & 255u) : 256u;
+            const uint32_t peers = __match_any_sync(kFull, bin);
+            if (hit && (peers & lanemask_lt()) == 0u) atomicAdd(&sm.hist[bin], static_cast<uint32_t>(__popc(peers)));
         }
-        __syncwarp();
-        uint32_t cnt[8];
-        uint32_t sum = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            cnt[e] = hist[lane * 8 + e];
-            sum += cnt[e];
-        }
-        uint32_t incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t v = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += v;
-        }
-        const uint32_t excl = incl - sum;
-        const bool here = excl < k_rem && k_rem <= incl;
-        const int src = __ffs(__ballot_sync(kFull, here)) - 1;
-        uint32_t digit = 0, below = 0;
-        if (here) {
-            uint32_t run = excl;
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t cnt[8];
+            uint32_t sum = 0;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                if (run + cnt[e] >= k_rem) {
-                    digit = static_cast<uint32_t>(lane * 8 + e);
-                    below = run;
-                    break;
+                cnt[e] = sm.hist[lane * 8 + e];
+                sum += cnt[e];
+            }
+            uint32_t incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t v = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const uint32_t excl = incl - sum;
+            if (excl < k_rem && k_rem <= incl) {  // exactly one lane holds the k-th key's digit
+                uint32_t run = excl;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if (run + cnt[e] >= k_rem) {
+                        sm.digit = static_cast<uint32_t>(lane * 8 + e);
+                        sm.below = run;
+                        break;
+                    }
+                    run += cnt[e];
                 }
-                run += cnt[e];
             }
         }
-        digit = __shfl_sync(kFull, digit, src);
-        below = __shfl_sync(kFull, below, src);
-        k_rem -= below;
-        prefix |= digit << shift;
+        __syncthreads();
+        k_rem -= sm.below;
+        prefix |= sm.digit << shift;
         mask |= 255u << shift;
-        __syncwarp();
     }
-    k_eq = static_cast<int>(k_rem);
-    return prefix;
-}
+    if (warp != 0) return;
+    const uint32_t T = prefix;
+    const int k_eq = static_cast<int>(k_rem);  // keys equal to T that belong to the k smallest
 
-__global__ void __launch_bounds__(kThreads) draft_kernel(const DraftArgs a) {
-    __shared__ DraftSmem sm;
-    extern __shared__ uint32_t keys[];  // [kG][cand_cap]
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int groups_per_layer = (a.nblk + kG - 1) / kG;
-    int cta = blockIdx.x;
-    const int gi = cta % groups_per_layer;
-    cta /= groups_per_layer;
-    const int ql = cta % a.q_layers;
-    const int h = cta / a.q_layers;
-    const int qb = gi * kG + warp;  // this warp's query block (within its layer)
-    const bool has_block = qb < a.nblk;
-    const int unit = (h * a.q_layers + ql) * a.nblk + qb;  // its (head, query block) row
-
-    // ---- 1. block mean of q (warp w: query block w)
-    const int qby = has_block ? qb / a.grid_w : 0;
-    const int qbx = has_block ? qb - qby * a.grid_w : 0;
-    if (has_block) {
-        const size_t frame = static_cast<size_t>(h) * a.tq + ql * 2;
-        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll 1
-        for (int n0 = 0; n0 < kBlockTokens; n0 += 32) {
-            uint2 raw[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {  // tokens in (t, y, x) row-major order
-                const int n = n0 + i;
-                const int t = n >> 6, y = (n >> 3) & 7, x = n & 7;
-                const size_t tok = ((frame + t) * a.tok_h + qby * 8 + y) * a.tok_w + qbx * 8 + x;
-                raw[i] = __ldg(reinterpret_cast<const uint2 *>(a.q + tok * kHeadDim) + lane);
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                acc0 += __uint_as_float(raw[i].x << 16);
-                acc1 += __uint_as_float(raw[i].x & 0xFFFF0000u);
-                acc2 += __uint_as_float(raw[i].y << 16);
-                acc3 += __uint_as_float(raw[i].y & 0xFFFF0000u);
-            }
-        }
-        const float4 m = make_float4(acc0 * (1.0f / 128.0f), acc1 * (1.0f / 128.0f), acc2 * (1.0f / 128.0f),
-                                     acc3 * (1.0f / 128.0f));
-        reinterpret_cast<float4 *>(sm.mq[warp])[lane] = m;
-        if (a.qmean) reinterpret_cast<float4 *>(a.qmean + static_cast<size_t>(unit) * kHeadDim)[lane] = m;
-        if (lane == 0) {
-            int y0, y1, x0, x1;
-            window_1d(qby, a.grid_h, a.local_range, a.local_mode, y0, y1);
-            window_1d(qbx, a.grid_w, a.local_range, a.local_mode, x0, x1);
-            sm.win[warp][0] = y0;
-            sm.win[warp][1] = y1;
-            sm.win[warp][2] = x0;
-            sm.win[warp][3] = x1;
-        }
-    } else if (lane == 0) {
-        sm.win[warp][0] = -1;
-        sm.win[warp][1] = sm.win[warp][2] = sm.win[warp][3] = 0;
-    }
-    const int q_layer_abs = a.count - a.q_layers + ql;  // key layer of these query blocks
-    const int n_layers = q_layer_abs + 1;
-    const int n_keys = a.count * a.nblk;
-    float *srow = (a.scores && has_block) ? a.scores + static_cast<size_t>(unit) * n_keys : nullptr;
-    if (srow) {
-        for (int j = lane; j < n_keys; j += 32) srow[j] = -INFINITY;
-    }
-    __syncthreads();  // means, windows and the -inf prefill are visible to every warp
-
-    // union of the windows of the group (bounding box per layer)
-    int uy0 = a.grid_h, uy1 = 0, ux0 = a.grid_w, ux1 = 0;
-#pragma unroll
-    for (int r = 0; r < kG; ++r) {
-        if (sm.win[r][0] < 0) continue;
-        uy0 = min(uy0, sm.win[r][0]);
-        uy1 = max(uy1, sm.win[r][1]);
-        ux0 = min(ux0, sm.win[r][2]);
-        ux1 = max(ux1, sm.win[r][3]);
-    }
-    const int unx = ux1 - ux0;
-    const int uper = (uy1 - uy0) * unx;
-    const int ucnt = n_layers * uper;  // <= cand_cap
-
-    // ---- 2. scores: one union candidate per thread, its mean read once
-    for (int u = tid; u < ucnt; u += kThreads) {
-        const int layer = u / uper;
-        const int rem = u - layer * uper;
-        const int yy = uy0 + rem / unx;
-        const int xx = ux0 + rem - (rem / unx) * unx;
-        const int b = yy * a.grid_w + xx;
-        int slot = a.oldest + layer;
-        if (slot >= a.capacity) slot -= a.capacity;
-        const float4 *mk =
-            reinterpret_cast<const float4 *>(a.kmean + ((static_cast<size_t>(slot) * a.heads + h) * a.nblk + b) * kHeadDim);
-        bool in[kG];
-#pragma unroll
-        for (int r = 0; r < kG; ++r)
-            in[r] = sm.win[r][0] <= yy && yy < sm.win[r][1] && sm.win[r][2] <= xx && xx < sm.win[r][3];
-        float dot[kG];
-#pragma unroll
-        for (int r = 0; r < kG; ++r) dot[r] = 0.f;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {  // 16 independent 16-byte loads in flight
-            float4 kv[16];
-#pragma unroll
-            for (int d4 = 0; d4 < 16; ++d4) kv[d4] = __ldg(mk + half * 16 + d4);
-#pragma unroll
-            for (int r = 0; r < kG; ++r) {
-                if (!in[r]) continue;
-                const float4 *mq4 = reinterpret_cast<const float4 *>(sm.mq[r]) + half * 16;
-#pragma unroll
-                for (int d4 = 0; d4 < 16; ++d4) {
-                    const float4 qv = mq4[d4];
-                    dot[r] = fmaf(qv.x, kv[d4].x, dot[r]);
-                    dot[r] = fmaf(qv.y, kv[d4].y, dot[r]);
-                    dot[r] = fmaf(qv.z, kv[d4].z, dot[r]);
-                    dot[r] = fmaf(qv.w, kv[d4].w, dot[r]);
-                }
-            }
-        }
-        const int j = layer * a.nblk + b;
-#pragma unroll
-        for (int r = 0; r < kG; ++r) {
-            const float score = dot[r] * a.scale;
-            keys[r * a.cand_cap + u] = in[r] ? desc_key(score) : kNotCandidate;
-            if (in[r] && a.scores) {
-                const int ur = (h * a.q_layers + ql) * a.nblk + gi * kG + r;
-                a.scores[static_cast<size_t>(ur) * n_keys + j] = score;
-            }
-        }
-    }
-    __syncthreads();
-    if (!has_block) return;
-
-    // ---- 3. exact top-k of this warp's block, written in ascending key index
-    const uint32_t *mykeys = keys + warp * a.cand_cap;
-    const int ncand =
-        n_layers * (sm.win[warp][1] - sm.win[warp][0]) * (sm.win[warp][3] - sm.win[warp][2]);  // >= 1
-    const int k = min(a.topk, ncand);
-    int k_eq = 0;
-    const uint32_t T = radix_select(mykeys, ucnt, k, sm.hist[warp], lane, k_eq);
+    // kept set in ascending key index
     int32_t *out = a.kept_idx + static_cast<size_t>(unit) * a.topk;
     const uint32_t lt_mask = lanemask_lt();
     int out_pos = 0, eq_seen = 0;
-    for (int base_u = 0; base_u < ucnt; base_u += 32) {
-        const int u = base_u + lane;
-        const uint32_t key = u < ucnt ? mykeys[u] : kNotCandidate;
-        const bool valid = key != kNotCandidate;
+    for (int base = 0; base < ncand; base += 32) {
+        const int c = base + lane;
+        const bool valid = c < ncand;
+        const uint32_t key = valid ? keys[c] : 0xFFFFFFFFu;
         const bool eq = valid && key == T;
         const uint32_t eqb = __ballot_sync(kFull, eq);
         const int eq_rank = eq_seen + __popc(eqb & lt_mask);
         const bool take = valid && (key < T || (eq && eq_rank < k_eq));
         const uint32_t tb = __ballot_sync(kFull, take);
         if (take) {
-            const int layer = u / uper;
-            const int rem = u - layer * uper;
-            const int yy = uy0 + rem / unx;
-            const int xx = ux0 + rem - (rem / unx) * unx;
-            out[out_pos + __popc(tb & lt_mask)] = layer * a.nblk + yy * a.grid_w + xx;
+            const int layer = div_by(c, m_wsz);
+            const int rem = c - layer * wsz;
+            const int ry = div_by(rem, m_wx);
+            out[out_pos + __popc(tb & lt_mask)] = layer * a.nblk + (y0 + ry) * a.grid_w + x0 + rem - ry * wx;
         }
         out_pos += __popc(tb);
         eq_seen += __popc(eqb);
@@ -304,14 +315,14 @@ __global__ void __launch_bounds__(kThreads) draft_kernel(const DraftArgs a) {
 }  // namespace
 
 cudaError_t launch_draft(const DraftArgs &a, cudaStream_t stream) {
-    const int groups = a.heads * a.q_layers * ((a.nblk + kG - 1) / kG);
-    const size_t smem = static_cast<size_t>(kG) * 4 * static_cast<size_t>(a.cand_cap);
+    const int rows = a.heads * a.q_layers * a.nblk;
+    const size_t smem = 4 * static_cast<size_t>(a.cand_cap);
     if (smem > 48 * 1024 - sizeof(DraftSmem)) {
         cudaError_t e = cudaFuncSetAttribute(draft_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
-    draft_kernel<<<groups, kThreads, smem, stream>>>(a);
+    draft_kernel<<<rows, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 

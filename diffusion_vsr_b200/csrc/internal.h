@@ -40,7 +40,7 @@ struct DraftArgs {
     int32_t heads, grid_h, grid_w, nblk, q_layers, tq, tok_h, tok_w;
     int32_t capacity, oldest, count;
     int32_t local_range, local_mode, topk;
-    int32_t cand_cap;      // candidates of the widest 8-block group union, rounded up to 32
+    int32_t cand_cap;      // most allowed candidates of a row, rounded up to 32
     float scale;
     int32_t *kept_idx;
     int32_t *kept_cnt;

@@ -91,44 +91,6 @@ int64_t max_candidates(const lcsa_params *p, const lcsa_kv_cache *c) {
     return static_cast<int64_t>(c->count) * span(p->grid_h) * span(p->grid_w);
 }
 
-// Allowed block range [lo, hi) along one axis (same rule as the draft kernel).
-void window_1d(int i, int n, int r, int mode, int &lo, int &hi) {
-    if (r <= 0 || (mode == 0 && n <= r)) {
-        lo = 0;
-        hi = n;
-        return;
-    }
-    const int h = r / 2;
-    if (mode == 0) {
-        lo = std::min(std::max(i - h, 0), n - r);
-        hi = lo + r;
-    } else {
-        lo = std::max(i - h, 0);
-        hi = std::min(i + h + 1, n);
-    }
-}
-
-// Largest union of the windows of 8 consecutive query blocks (the draft
-// kernel scores such a union once per group), times the key layers.
-int64_t max_group_union(const lcsa_params *p, const lcsa_kv_cache *c) {
-    const int nblk = p->grid_h * p->grid_w;
-    int64_t best = 0;
-    for (int g0 = 0; g0 < nblk; g0 += 8) {
-        int uy0 = p->grid_h, uy1 = 0, ux0 = p->grid_w, ux1 = 0;
-        for (int qb = g0; qb < std::min(g0 + 8, nblk); ++qb) {
-            int y0, y1, x0, x1;
-            window_1d(qb / p->grid_w, p->grid_h, p->local_range, p->local_mode, y0, y1);
-            window_1d(qb % p->grid_w, p->grid_w, p->local_range, p->local_mode, x0, x1);
-            uy0 = std::min(uy0, y0);
-            uy1 = std::max(uy1, y1);
-            ux0 = std::min(ux0, x0);
-            ux1 = std::max(ux1, x1);
-        }
-        best = std::max<int64_t>(best, static_cast<int64_t>(uy1 - uy0) * (ux1 - ux0));
-    }
-    return best * c->count;
-}
-
 // Rank-4 map over a token-layout bf16 tensor [H*T][8gh][8gw][128] with a
 // (64 dims, 8, 8, 2 frames) box and 128-byte swizzle: one box pair is one
 // (2,8,8) window block, so the partition is done by the copy engine.
@@ -244,7 +206,7 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
     a.local_range = p->local_range;
     a.local_mode = p->local_mode;
     a.topk = p->topk;
-    a.cand_cap = static_cast<int32_t>((max_group_union(p, cache) + 31) / 32 * 32);
+    a.cand_cap = static_cast<int32_t>((cand + 31) / 32 * 32);
     a.scale = eff_scale(p);
     a.kept_idx = kept_idx;
     a.kept_cnt = kept_cnt;
