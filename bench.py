@@ -353,7 +353,10 @@ def oracle_chunk_sample(w: W.Workload, rows_sample: int, seed: int = 0):
     t1 = time.perf_counter()
     rng = np.random.default_rng(seed)
     Nq = w.n_query_blocks
-    rows = [(int(rng.integers(w.heads)), int(rng.integers(Nq))) for _ in range(rows_sample)]
+    if rows_sample >= w.heads * Nq:  # every row of the chunk
+        rows = [(h, i) for h in range(w.heads) for i in range(Nq)]
+    else:
+        rows = [(int(rng.integers(w.heads)), int(rng.integers(Nq))) for _ in range(rows_sample)]
     qb = O.partition(qf)
     kb, vb = oc.keys()
     scale = 1 / np.sqrt(128.0)
@@ -361,7 +364,7 @@ def oracle_chunk_sample(w: W.Workload, rows_sample: int, seed: int = 0):
         O.sparse_attention_row(qb[h, i], kb[h], vb[h], res["kept_idx"][h, i, :res["kept_cnt"][h, i]], scale)
     t2 = time.perf_counter()
     total_rows = w.heads * Nq
-    est = (t1 - t0) + (t2 - t1) * total_rows / max(1, rows_sample)
+    est = (t1 - t0) + (t2 - t1) * total_rows / max(1, len(rows))
     kept_tiles = int(res["kept_cnt"].sum())
     return {"measured_s": t2 - t0, "chunk_s_est": est, "kept_tiles": kept_tiles,
             "sample": f"one chunk: full append+draft ({total_rows} rows) + attention on {rows_sample} of "
@@ -379,12 +382,23 @@ def cpu_cores() -> int:
     return len(os.sched_getaffinity(0))
 
 
-def cpu_baseline(w: W.Workload, rows_sample: int = 48):
-    r = oracle_chunk_sample(w, rows_sample)
-    value = r["kept_tiles"] * W.flops_per_tile() / r["chunk_s_est"] / 1e12
+def cpu_baseline(w: W.Workload, target_s: float = 10.0, max_chunks: int = 4):
+    """The oracle on whole chunks (append, draft and attention of every row),
+    repeated on successive seeds until about ``target_s`` seconds of CPU work."""
+    total_rows = w.heads * w.n_query_blocks
+    spent, est, kept, n = 0.0, 0.0, 0, 0
+    while n < max_chunks and (n == 0 or spent < target_s):
+        r = oracle_chunk_sample(w, total_rows, seed=n)
+        spent += r["measured_s"]
+        est += r["chunk_s_est"]
+        kept += r["kept_tiles"]
+        n += 1
+    value = kept * W.flops_per_tile() / est / 1e12
     return {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-            "ms_per_chunk": round(r["chunk_s_est"] * 1e3, 1), "sample": r["sample"],
-            "measured_s": round(r["measured_s"], 2)}
+            "ms_per_chunk": round(est / n * 1e3, 1),
+            "sample": f"{n} x one whole chunk: append + draft + attention of all {total_rows} rows, "
+                      f"fp64 NumPy oracle",
+            "measured_s": round(spent, 2)}
 
 
 def run_reference(args):
