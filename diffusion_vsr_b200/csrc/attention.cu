@@ -31,8 +31,9 @@
 //                  query row per thread, online softmax in the log2 domain with
 //                  lazy rescaling of O (only when the row maximum grew by more
 //                  than 2^8), P written as bf16 over S.  At the end of a row both
-//                  groups merge (m, l, O) and each writes one 64-dim half of the
-//                  bf16 output straight into token layout (reverse partition).
+//                  groups merge (m, l, O); each stages one 64-dim half of the
+//                  bf16 output tile in the row's Q buffer and writes it with one
+//                  TMA store into token layout (the reverse partition).
 // TMEM (512 columns): S_w at 128*w, O_w at 256 + 128*w.
 // Every wait is bounded; on expiry the CTA drains its copies and MMAs, frees
 // TMEM and reports LCSA_ERR_TIMEOUT.
@@ -187,7 +188,8 @@ __device__ __forceinline__ bool issue_pv(AttnSmem &sm, const MmaCtx &m, int w, i
 
 __global__ void __launch_bounds__(kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const AttnArgs a, uint16_t *__restrict__ out) {
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                     const AttnArgs a, uint16_t *__restrict__ out) {
     extern __shared__ uint8_t smem_raw[];
     AttnSmem &sm = *reinterpret_cast<AttnSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                   ~static_cast<uintptr_t>(1023));
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&sm.bar_qfull[b]), 1);
-            mbar_init(smem_u32(&sm.bar_qempty[b]), 8);  // one arrival per softmax warp
+            mbar_init(smem_u32(&sm.bar_qempty[b]), 2);  // one arrival per softmax group (its output copy read the buffer)
             mbar_init(smem_u32(&sm.bar_sfull[b]), 1);
             for (int qq = 0; qq < 4; ++qq) mbar_init(smem_u32(&sm.bar_pq[qq][b]), 4);  // one arrival per warp
             mbar_init(smem_u32(&sm.bar_drain[b]), 1);
@@ -224,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_o);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
@@ -516,7 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float L = l * a_self + l_o * a_oth;
             const float inv_l = L > 0.f ? 1.f / L : 0.f;
             const float f_self = a_self * inv_l, f_oth = a_oth * inv_l;
-            // this group writes output dims [64w, 64w+64) of its row
+            // this group's output dims [64w, 64w+64) of its row, merged and packed to bf16
+            uint32_t pk[2][16];
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const uint32_t col = static_cast<uint32_t>(w * 64 + cc * 32);
@@ -534,27 +538,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int k = 0; k < 32; ++k) o1[k] = 0u;
                 }
                 tmem_wait_ld();
-                uint32_t pk[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     const float x0 = __uint_as_float(o0[2 * k]) * f_self + __uint_as_float(o1[2 * k]) * f_oth;
                     const float x1 = __uint_as_float(o0[2 * k + 1]) * f_self + __uint_as_float(o1[2 * k + 1]) * f_oth;
-                    pk[k] = pack_bf16x2(x0, x1);
+                    pk[cc][k] = pack_bf16x2(x0, x1);
                 }
-#pragma unroll
-                for (int qd = 0; qd < 4; ++qd)
-                    dst[cc * 4 + qd] = make_uint4(pk[4 * qd], pk[4 * qd + 1], pk[4 * qd + 2], pk[4 * qd + 3]);
             }
-            if (w == 0 && a.lse) a.lse[tok] = L > 0.f ? (m + __log2f(L)) * kLn2 : -INFINITY;
-            // O of both groups and this Q buffer (the exchange) are free again
+            // O of both groups has been read: the next row's PVs may overwrite it
             tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ofree));
+            if (w == 0 && a.lse) a.lse[tok] = L > 0.f ? (m + __log2f(L)) * kLn2 : -INFINITY;
+            // every thread has read the (m, l) exchange before the tile overwrites it
             named_bar_sync(3, 256);
-            if (lane == 0) {
-                mbar_arrive(smem_u32(&sm.bar_ofree));
+            // Stage this group's half of the bf16 output tile in the row's Q buffer,
+            // 128-byte swizzled as the TMA box expects (row = token of the block,
+            // 16-byte chunk c of the row at chunk position c ^ (row & 7)), then one
+            // TMA store per group writes it into token layout (reverse partition).
+            uint8_t *half_buf = sm.q[qb] + w * kHalfBytes;
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+                for (int qd = 0; qd < 4; ++qd) {
+                    const int chunk = cc * 4 + qd;
+                    *reinterpret_cast<uint4 *>(half_buf + row * 128 + ((chunk ^ (row & 7)) << 4)) =
+                        make_uint4(pk[cc][4 * qd], pk[cc][4 * qd + 1], pk[cc][4 * qd + 2], pk[cc][4 * qd + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            if (w == 0) named_bar_sync(4, 128);  // (constant ids: the barrier count stays known)
+            else named_bar_sync(5, 128);
+            if (quad == 0 && lane == 0) {
+                tma_store_4d(&tm_o, smem_u32(half_buf), 64 * w, rg.qbx * 8, rg.qby * 8, rg.frame0);
+                bulk_commit_group();
+                bulk_wait_group_read0();  // the Q buffer may be refilled once the copy has read it
                 mbar_arrive(smem_u32(&sm.bar_qempty[qb]));
             }
             ++act;
         }
+        // the output copies of this group have landed before the CTA exits
+        if (quad == 0 && lane == 0) bulk_wait_group0();
     }
 
     __syncthreads();
@@ -577,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                             const AttnArgs &a, void *out, cudaStream_t stream) {
+                             const CUtensorMap &tm_o, const AttnArgs &a, void *out, cudaStream_t stream) {
     const size_t smem = sizeof(AttnSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -586,7 +610,7 @@ cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, c
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const int grid = a.n_units < sms ? a.n_units : sms;
-    attention_kernel<<<grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, a, static_cast<uint16_t *>(out));
+    attention_kernel<<<grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, tm_o, a, static_cast<uint16_t *>(out));
     return cudaGetLastError();
 }
 

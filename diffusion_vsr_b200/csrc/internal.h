@@ -31,7 +31,7 @@ struct AttnArgs {
 };
 
 cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                             const AttnArgs &a, void *out, cudaStream_t stream);
+                             const CUtensorMap &tm_o, const AttnArgs &a, void *out, cudaStream_t stream);
 
 // Draft mask: q block means, scores over allowed candidates, top-k.
 struct DraftArgs {

@@ -230,9 +230,9 @@ int lcsa_attention(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache 
     const int nblk = p->grid_h * p->grid_w;
     const int64_t frames = static_cast<int64_t>(p->heads) * 2 * p->q_layers;
     const int64_t rows = static_cast<int64_t>(cache->capacity) * cache->heads * nblk * kBlockTokens;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!make_token_map(&tq, q_tok, frames, 8 * p->grid_h, 8 * p->grid_w) || !make_ring_map(&tk, cache->k, rows) ||
-        !make_ring_map(&tv, cache->v, rows))
+        !make_ring_map(&tv, cache->v, rows) || !make_token_map(&to, out_tok, frames, 8 * p->grid_h, 8 * p->grid_w))
         return LCSA_ERR_CUDA;
 
     lcsa::AttnArgs a{};
@@ -256,7 +256,7 @@ int lcsa_attention(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache 
     a.status = d_status;
     a.timeout_ns = lcsa::kWatchdogNs;
     a.flags = p->flags;
-    if (lcsa::launch_attention(tq, tk, tv, a, out_tok, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (lcsa::launch_attention(tq, tk, tv, to, a, out_tok, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LCSA_ERR_CUDA;
     return LCSA_OK;
 }
