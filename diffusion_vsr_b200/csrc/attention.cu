@@ -89,19 +89,30 @@ struct __align__(1024) AttnSmem {
 __device__ __forceinline__ uint32_t col_s(int w) { return static_cast<uint32_t>(w) * 128u; }
 __device__ __forceinline__ uint32_t col_o(int w) { return 256u + static_cast<uint32_t>(w) * 128u; }
 
-// Kept tiles of a row, or 0 when its count or an index is out of range (whole warp).
-__device__ __forceinline__ int row_tiles(const AttnArgs &a, int unit, int lane, bool &bad) {
-    const int cnt = a.kept_cnt[unit];
+// Kept tiles of a row, or 0 when its count or an index is out of range (whole
+// warp).  cnt and idx0 (kept index number `lane` of the row) were prefetched.
+__device__ __forceinline__ int row_tiles(const AttnArgs &a, int unit, int cnt, int idx0, int lane, bool &bad) {
     bad = cnt < 0 || cnt > a.topk;
     if (!bad) {
+        if (lane < cnt) bad = idx0 < 0 || idx0 >= a.n_key_blocks;
         const int32_t *row = a.kept_idx + static_cast<size_t>(unit) * a.topk;
-        for (int i = lane; i < cnt; i += 32) {
+        for (int i = lane + 32; i < cnt; i += 32) {
             const int j = row[i];
             bad |= (j < 0 || j >= a.n_key_blocks);
         }
     }
     bad = __any_sync(0xffffffffu, bad);
     return bad ? 0 : cnt;
+}
+
+// Count and first 32 kept indices of row u (lane l: index l), or zeros past the end.
+__device__ __forceinline__ void fetch_row(const AttnArgs &a, int u, int lane, int &cnt, int &idx) {
+    cnt = 0;
+    idx = 0;
+    if (u < a.n_units) {
+        cnt = __ldg(a.kept_cnt + u);
+        if (lane < a.topk) idx = __ldg(a.kept_idx + static_cast<size_t>(u) * a.topk + lane);
+    }
 }
 
 struct RowGeom {
@@ -245,12 +256,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------------- producer
         // The whole warp walks the rows: it validates each kept list, publishes
         // the row's tile count to the consumers, and reads the kept indices 32 at
-        // a time (one coalesced load, then shuffles); lane 0 issues the copies.
+        // a time (one coalesced load, then shuffles; the count and the first 32
+        // indices of the next row are loaded one row ahead); lane 0 issues the
+        // copies.
         int g = 0, act = 0, r = 0;  // tiles, non-empty rows and rows so far
         bool ok = true;
+        int cnt_next, idx_next;  // the next row's kept list, loaded one row ahead
+        fetch_row(a, blockIdx.x, lane, cnt_next, idx_next);
         for (int unit = blockIdx.x; unit < a.n_units; unit += gridDim.x, ++r) {
+            const int cnt = cnt_next, idx0 = idx_next;
+            fetch_row(a, unit + gridDim.x, lane, cnt_next, idx_next);
             bool bad;
-            const int n = row_tiles(a, unit, lane, bad);
+            const int n = row_tiles(a, unit, cnt, idx0, lane, bad);
             if (lane == 0) {
                 if (bad && a.status) atomicOr(a.status, LCSA_ERR_BAD_INDEX);
                 const int is = r % kInfoSlots;
@@ -281,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int32_t *kept_row = a.kept_idx + static_cast<size_t>(unit) * a.topk;
             int idx = 0;
             for (int j = 0; ok && j < n; ++j) {
-                if ((j & 31) == 0) idx = (j + lane < n) ? __ldg(kept_row + j + lane) : 0;
+                if ((j & 31) == 0) idx = j == 0 ? idx0 : ((j + lane < n) ? __ldg(kept_row + j + lane) : 0);
                 const int kb = __shfl_sync(0xffffffffu, idx, j & 31);
                 if (lane == 0) {
                     const int gk = g + j;
@@ -393,6 +410,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tok_t = row >> 6, tok_y = (row >> 3) & 7, tok_x = row & 7;  // token of this row
         int act = 0, t = 0, r = 0;
         bool ok = true;
+        // One thread per group issues the group's output copies.  The Q buffer
+        // a copy reads from is handed back to the producer (bar_qempty) only
+        // once the copy has read it, which is checked later, when it has long
+        // completed, rather than waited for.
+        const bool elected = quad == 0 && lane == 0;
+        int pending_q = -1;
+        auto release_q = [&](int b) {
+            bulk_wait_group_read0();
+            mbar_arrive(smem_u32(&sm.bar_qempty[b]));
+            pending_q = -1;
+        };
         for (int unit = blockIdx.x; unit < a.n_units; unit += gridDim.x, ++r) {
             const int is = r % kInfoSlots;
             ok = __all_sync(0xffffffffu,
@@ -498,6 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
                 l = l * alpha + rs;
                 m_used = m_next;
+                if (i == 0 && elected && pending_q >= 0) release_q(pending_q);
             }
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_ofinal), act & 1, abort_word, to));
             // both groups take the same decision on going through the epilogue
@@ -569,16 +598,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             if (w == 0) named_bar_sync(4, 128);  // (constant ids: the barrier count stays known)
             else named_bar_sync(5, 128);
-            if (quad == 0 && lane == 0) {
+            if (elected) {
+                if (pending_q >= 0) release_q(pending_q);
                 tma_store_4d(&tm_o, smem_u32(half_buf), 64 * w, rg.qbx * 8, rg.qby * 8, rg.frame0);
                 bulk_commit_group();
-                bulk_wait_group_read0();  // the Q buffer may be refilled once the copy has read it
-                mbar_arrive(smem_u32(&sm.bar_qempty[qb]));
+                pending_q = qb;  // released once the copy has read it (next row's first tile)
             }
             ++act;
         }
         // the output copies of this group have landed before the CTA exits
-        if (quad == 0 && lane == 0) bulk_wait_group0();
+        if (elected) {
+            if (pending_q >= 0) release_q(pending_q);
+            bulk_wait_group0();
+        }
     }
 
     __syncthreads();
