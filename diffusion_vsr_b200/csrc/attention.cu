@@ -119,14 +119,18 @@ struct RowGeom {
     int h, ql, qby, qbx, frame0;
 };
 
+__device__ __forceinline__ int mul_div(int n, uint64_t m) {
+    return static_cast<int>((static_cast<uint64_t>(static_cast<uint32_t>(n)) * m) >> 32);
+}
+
 __device__ __forceinline__ RowGeom row_geom(const AttnArgs &a, int unit) {
     RowGeom g;
     const int nq = a.q_layers * a.nblk;
-    g.h = unit / nq;
+    g.h = mul_div(unit, a.m_nq);
     const int qi = unit - g.h * nq;
-    g.ql = qi / a.nblk;
+    g.ql = mul_div(qi, a.m_nblk);
     const int qb = qi - g.ql * a.nblk;
-    g.qby = qb / a.grid_w;
+    g.qby = mul_div(qb, a.m_gw);
     g.qbx = qb - g.qby * a.grid_w;
     g.frame0 = g.h * a.tq + g.ql * 2;  // first frame of the block in the Q/O maps
     return g;
@@ -302,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int kb = __shfl_sync(0xffffffffu, idx, j & 31);
                 if (lane == 0) {
                     const int gk = g + j;
-                    const int layer = kb / a.nblk;
+                    const int layer = mul_div(kb, a.m_nblk);
                     const int b = kb - layer * a.nblk;
                     int slot = a.oldest + layer;
                     if (slot >= a.capacity) slot -= a.capacity;
@@ -550,28 +554,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float f_self = a_self * inv_l, f_oth = a_oth * inv_l;
             // this group's output dims [64w, 64w+64) of its row, merged and packed to bf16
             uint32_t pk[2][16];
+            {
+                // both 32-column halves of both accumulators in one TMEM round trip
+                uint32_t o0[2][32], o1[2][32];
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const uint32_t col = static_cast<uint32_t>(w * 64 + cc * 32);
-                uint32_t o0[32], o1[32];
-                if (n_mine > 0) {
-                    tmem_ld32(tmem + lane_off + col_o(w) + col, o0);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) o0[k] = 0u;
-                }
-                if (n_other > 0) {
-                    tmem_ld32(tmem + lane_off + col_o(1 - w) + col, o1);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) o1[k] = 0u;
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint32_t col = static_cast<uint32_t>(w * 64 + cc * 32);
+                    // (an accumulator without tiles holds stale data: selected away below)
+                    tmem_ld32(tmem + lane_off + col_o(w) + col, o0[cc]);
+                    tmem_ld32(tmem + lane_off + col_o(1 - w) + col, o1[cc]);
                 }
                 tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float x0 = __uint_as_float(o0[2 * k]) * f_self + __uint_as_float(o1[2 * k]) * f_oth;
-                    const float x1 = __uint_as_float(o0[2 * k + 1]) * f_self + __uint_as_float(o1[2 * k + 1]) * f_oth;
-                    pk[cc][k] = pack_bf16x2(x0, x1);
+                for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float a0 = n_mine > 0 ? __uint_as_float(o0[cc][2 * k]) : 0.f;
+                        const float a1 = n_mine > 0 ? __uint_as_float(o0[cc][2 * k + 1]) : 0.f;
+                        const float b0 = n_other > 0 ? __uint_as_float(o1[cc][2 * k]) : 0.f;
+                        const float b1 = n_other > 0 ? __uint_as_float(o1[cc][2 * k + 1]) : 0.f;
+                        pk[cc][k] = pack_bf16x2(a0 * f_self + b0 * f_oth, a1 * f_self + b1 * f_oth);
+                    }
                 }
             }
             // O of both groups has been read: the next row's PVs may overwrite it

@@ -28,7 +28,13 @@ struct AttnArgs {
     int32_t *status;       // may be null
     uint64_t timeout_ns;
     int32_t flags;
+    // ceil(2^32 / d) for d = q_layers * nblk, nblk, grid_w: n / d = (n * m) >> 32
+    // exactly while n * d <= 2^32 (checked by the caller for every n used)
+    uint64_t m_nq, m_nblk, m_gw;
 };
+
+// Multiplier of the exact multiply-high division by d (1 <= d).
+inline uint64_t div_magic_host(uint32_t d) { return ((1ull << 32) + d - 1) / d; }
 
 cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                              const CUtensorMap &tm_o, const AttnArgs &a, void *out, cudaStream_t stream);

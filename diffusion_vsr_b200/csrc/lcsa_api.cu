@@ -256,6 +256,13 @@ int lcsa_attention(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache 
     a.status = d_status;
     a.timeout_ns = lcsa::kWatchdogNs;
     a.flags = p->flags;
+    // multiply-high division stays exact while every dividend times its divisor is <= 2^32
+    const int64_t nq = static_cast<int64_t>(p->q_layers) * nblk;
+    if (static_cast<int64_t>(a.n_units) * nq > (1ll << 32) || static_cast<int64_t>(a.n_key_blocks) * nblk > (1ll << 32))
+        return LCSA_ERR_INVALID_ARG;
+    a.m_nq = lcsa::div_magic_host(static_cast<uint32_t>(nq));
+    a.m_nblk = lcsa::div_magic_host(static_cast<uint32_t>(nblk));
+    a.m_gw = lcsa::div_magic_host(static_cast<uint32_t>(p->grid_w));
     if (lcsa::launch_attention(tq, tk, tv, to, a, out_tok, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LCSA_ERR_CUDA;
     return LCSA_OK;
