@@ -76,45 +76,81 @@ def run_stream(w: W.Workload, n_steps: Optional[int] = None, n_rows: Optional[in
         _, k, v = W.gen_layers(w, p, 1, "kv")
         layer.append(k.to(dev), v.to(dev))
         ocache.append(f32(k), f32(v))
-    Nq = w.n_query_blocks
     results = []
     for p in steps[: (n_steps or len(steps))]:
         q, k, v = W.gen_layers(w, p, w.q_layers)
-        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-        L.lcsa_cache_append(layer.cache, kd, vd, d_status=layer.status)
-        ocache.append(f32(k), f32(v))
-        ring_ok = None
-        kmean_err = None
-        if check_ring:
-            ring_ok, kmean_err = ring_matches(layer.cache, ocache)
-        Nk = layer.cache.count * w.blocks_per_layer
-        scores = torch.empty((w.heads, Nq, Nk), dtype=torch.float32, device=dev)
-        qmean = torch.empty((w.heads, Nq, 128), dtype=torch.float32, device=dev)
-        L.lcsa_draft_mask(layer.params, qd, layer.cache, layer.kept_idx, layer.kept_cnt, scores, qmean,
-                          d_status=layer.status)
-        out_p = torch.empty_like(qd)
-        L.lcsa_attention(layer.params, qd, layer.cache, layer.kept_idx, layer.kept_cnt, out_p,
-                         d_status=layer.status)
-        # oracle draft + selection on every row; attention on sampled rows
-        rows = None if n_rows is None else sample_rows(w.heads, Nq, n_rows, seed_rows + p)
-        ref = O.lcsa_step(f32(q), ocache, w.grid_h, w.grid_w, w.topk, w.local_range, MODES[w.local_mode],
-                          rows=rows if rows is not None else [(h, i) for h in range(w.heads) for i in range(Nq)])
-        kept_o = torch.from_numpy(ref["kept_idx"]).to(dev)
-        cnt_o = torch.from_numpy(ref["kept_cnt"]).to(dev)
-        out_o = torch.empty_like(qd)
-        lse_o = torch.empty(qd.shape[:4], dtype=torch.float32, device=dev)
-        L.lcsa_attention(layer.params, qd, layer.cache, kept_o, cnt_o, out_o, lse_o, d_status=layer.status)
-        torch.cuda.synchronize()
-        exempt = O.near_tie_rows(ref["scores"], ref["allowed"], ref["mq"], ref["mk"], w.topk, NEAR_TIE_REL)
-        results.append(StepResult(
-            position=p, oracle=ref,
-            gpu_kept=layer.kept_idx.cpu().numpy(), gpu_cnt=layer.kept_cnt.cpu().numpy(),
-            gpu_scores=scores.cpu().numpy(), gpu_qmean=qmean.cpu().numpy(),
-            out_pipeline=O.partition(f32(out_p)), out_oracle_mask=O.partition(f32(out_o)),
-            lse_oracle_mask=O.partition(lse_o.cpu().numpy()[..., None])[..., 0],
-            rows=rows if rows is not None else [(h, i) for h in range(w.heads) for i in range(Nq)],
-            exempt=exempt, status=int(layer.status.item()), ring_ok=ring_ok, kmean_err=kmean_err))
+        results.append(step_both(w, layer.cache, ocache, layer.params, q, k, v, n_rows, check_ring,
+                                 seed_rows + p, p, layer.status))
     return results
+
+
+def run_schedule(w: W.Workload, schedule: List[int], n_rows: Optional[int] = None,
+                 check_ring: bool = False) -> List[StepResult]:
+    """A stream that starts from an empty cache of kv_len + 1 slots and appends
+    ``schedule[i]`` block-layers at step i (e.g. a cold-start chunk of 3 layers,
+    then chunks of 1), each step querying exactly the layers it appended."""
+    from diffusion_vsr_b200 import lcsa as L
+
+    dev = torch.device("cuda")
+    capacity = w.kv_len + 1
+    assert max(schedule) <= capacity
+    cache = L.KVCache.allocate(capacity, w.heads, w.grid_h, w.grid_w, dev)
+    ocache = O.KVCacheModel(capacity)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    results = []
+    pos = 0
+    for n_layers in schedule:
+        params = L.make_params(w.heads, w.grid_h, w.grid_w, n_layers, w.topk, w.local_range, w.local_mode)
+        q, k, v = W.gen_layers(w, pos, n_layers)
+        results.append(step_both(w, cache, ocache, params, q, k, v, n_rows, check_ring, pos, pos, status))
+        pos += n_layers
+    return results
+
+
+def step_both(w: W.Workload, cache, ocache: O.KVCacheModel, params, q, k, v, n_rows, check_ring, seed,
+              position, status) -> StepResult:
+    """Append one chunk, then draft + attention on the GPU (own mask and the
+    oracle's mask) and the oracle step on the same inputs."""
+    from diffusion_vsr_b200 import lcsa as L
+
+    dev = torch.device("cuda")
+    q_layers = q.shape[1] // 2
+    Nq = q_layers * w.blocks_per_layer
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    L.lcsa_cache_append(cache, kd, vd, d_status=status)
+    ocache.append(f32(k), f32(v))
+    ring_ok = None
+    kmean_err = None
+    if check_ring:
+        ring_ok, kmean_err = ring_matches(cache, ocache)
+    Nk = cache.count * w.blocks_per_layer
+    kept = torch.empty((w.heads, Nq, w.topk), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.heads, Nq), dtype=torch.int32, device=dev)
+    scores = torch.empty((w.heads, Nq, Nk), dtype=torch.float32, device=dev)
+    qmean = torch.empty((w.heads, Nq, 128), dtype=torch.float32, device=dev)
+    L.lcsa_draft_mask(params, qd, cache, kept, cnt, scores, qmean, d_status=status)
+    out_p = torch.empty_like(qd)
+    L.lcsa_attention(params, qd, cache, kept, cnt, out_p, d_status=status)
+    # oracle draft + selection on every row; attention on sampled rows
+    rows = None if n_rows is None else sample_rows(w.heads, Nq, n_rows, seed)
+    all_rows = [(h, i) for h in range(w.heads) for i in range(Nq)]
+    ref = O.lcsa_step(f32(q), ocache, w.grid_h, w.grid_w, w.topk, w.local_range, MODES[w.local_mode],
+                      rows=rows if rows is not None else all_rows)
+    kept_o = torch.from_numpy(ref["kept_idx"]).to(dev)
+    cnt_o = torch.from_numpy(ref["kept_cnt"]).to(dev)
+    out_o = torch.empty_like(qd)
+    lse_o = torch.empty(qd.shape[:4], dtype=torch.float32, device=dev)
+    L.lcsa_attention(params, qd, cache, kept_o, cnt_o, out_o, lse_o, d_status=status)
+    torch.cuda.synchronize()
+    exempt = O.near_tie_rows(ref["scores"], ref["allowed"], ref["mq"], ref["mk"], w.topk, NEAR_TIE_REL)
+    return StepResult(
+        position=position, oracle=ref,
+        gpu_kept=kept.cpu().numpy(), gpu_cnt=cnt.cpu().numpy(),
+        gpu_scores=scores.cpu().numpy(), gpu_qmean=qmean.cpu().numpy(),
+        out_pipeline=O.partition(f32(out_p)), out_oracle_mask=O.partition(f32(out_o)),
+        lse_oracle_mask=O.partition(lse_o.cpu().numpy()[..., None])[..., 0],
+        rows=rows if rows is not None else all_rows,
+        exempt=exempt, status=int(status.item()), ring_ok=ring_ok, kmean_err=kmean_err)
 
 
 def ring_matches(cache, ocache: O.KVCacheModel) -> Tuple[bool, float]:

@@ -116,6 +116,33 @@ def test_truncated_window_ragged_counts():
     _check_step(res, w)
 
 
+def test_cold_start_three_layers_then_streaming():
+    # The first chunk of a stream carries 3 block-layers (6 latent frames) into
+    # an empty cache; the next chunks carry 1 layer each and see the cached
+    # ones, the oldest dropped once kv_len + 1 slots are full.
+    w = W.WORKLOADS["768x1280"]
+    results = Hn.run_schedule(w, [3, 1, 1], n_rows=24, check_ring=True)
+    nb = w.blocks_per_layer
+    first = results[0]
+    # block-causal inside the chunk: query layer L allows the keys of layers 0..L
+    allowed = first.oracle["allowed"].sum(axis=1)
+    assert np.array_equal(allowed, np.repeat([nb, 2 * nb, 3 * nb], nb))
+    assert [r.oracle["allowed"].shape[1] for r in results] == [3 * nb, 4 * nb, 4 * nb]
+    for res in results:
+        assert res.ring_ok and res.kmean_err <= 1e-6
+        _check_step(res, w)
+
+
+def test_global_window_1536x2688():
+    # local_range <= 0: no local window (every key block of the visible layers
+    # is a candidate), the per-layer alternative a hybrid local/global stack uses
+    import dataclasses
+    w = dataclasses.replace(W.WORKLOADS["1536x2688"], local_range=0)
+    (res,) = Hn.run_stream(w, n_steps=1, n_rows=12)
+    assert res.oracle["allowed"].sum(axis=1).min() == w.capacity * w.blocks_per_layer
+    _check_step(res, w)
+
+
 def test_deterministic_byte_identical():
     w = W.WORKLOADS["768x1280"]
     a = Hn.run_stream(w, n_rows=4)[0]
