@@ -195,3 +195,67 @@ class LcsaLayer:
         lcsa_draft_mask(self.params, q_tok, self.cache, self.kept_idx, self.kept_cnt, d_status=self.status)
         lcsa_attention(self.params, q_tok, self.cache, self.kept_idx, self.kept_cnt, out_tok, lse,
                        d_status=self.status)
+
+
+class HostStream:
+    """Host-fed streaming over an :class:`LcsaLayer` with copies overlapped.
+
+    Chunk i's q/k/v are copied from pinned host memory on a copy stream while
+    chunk i-1 computes, and chunk i-1's output is copied back on a second copy
+    stream while chunk i computes: two device slots per buffer, ordered by
+    CUDA events (no host synchronisation).  Each ``submit`` enqueues one chunk
+    (append + draft + attention through the C ABI) and returns at once; the
+    host output buffer of chunk i is complete once ``done(i)`` is.
+    """
+
+    def __init__(self, layer: LcsaLayer, q_shape, device="cuda", depth: int = 2):
+        self.layer = layer
+        self.device = torch.device(device)
+        self.depth = depth
+        self.compute = torch.cuda.current_stream(self.device)
+        self.copy_in = torch.cuda.Stream(self.device)
+        self.copy_out = torch.cuda.Stream(self.device)
+        mk = lambda: torch.empty(q_shape, dtype=torch.bfloat16, device=self.device)
+        self.inputs = [(mk(), mk(), mk()) for _ in range(depth)]
+        self.outputs = [mk() for _ in range(depth)]
+        ev = lambda: torch.cuda.Event()
+        self.in_ready = [ev() for _ in range(depth)]
+        self.computed = [ev() for _ in range(depth)]
+        self.copied_out = [ev() for _ in range(depth)]
+        for e in self.computed + self.copied_out:  # every slot starts free
+            e.record(self.compute)
+        self._n = 0
+
+    def submit(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor,
+               out_host: torch.Tensor) -> int:
+        i = self._n
+        b = i % self.depth
+        q, k, v = self.inputs[b]
+        # copy in once the chunk that last used this slot finished computing
+        self.copy_in.wait_event(self.computed[b])
+        with torch.cuda.stream(self.copy_in):
+            q.copy_(q_host, non_blocking=True)
+            k.copy_(k_host, non_blocking=True)
+            v.copy_(v_host, non_blocking=True)
+            self.in_ready[b].record(self.copy_in)
+        # compute once the inputs landed and the slot's previous output left
+        self.compute.wait_event(self.in_ready[b])
+        self.compute.wait_event(self.copied_out[b])
+        with torch.cuda.stream(self.compute):
+            self.layer.step(q, k, v, self.outputs[b])
+        self.computed[b].record(self.compute)
+        self.copy_out.wait_event(self.computed[b])
+        with torch.cuda.stream(self.copy_out):
+            out_host.copy_(self.outputs[b], non_blocking=True)
+            self.copied_out[b].record(self.copy_out)
+        self._n += 1
+        return i
+
+    def done(self, i: int) -> torch.cuda.Event:
+        """Event after which chunk i's output is in its host buffer (valid until chunk i + depth is submitted)."""
+        return self.copied_out[i % self.depth]
+
+    def drain_into(self, stream: torch.cuda.Stream) -> None:
+        """Make ``stream`` wait for every copy and computation submitted so far."""
+        for e in self.copied_out:
+            stream.wait_event(e)

@@ -152,6 +152,40 @@ def test_deterministic_byte_identical():
     assert np.array_equal(a.out_pipeline, b.out_pipeline)
 
 
+def test_host_stream_matches_direct_steps():
+    # Overlapped host streaming (copy in / compute / copy out on three streams)
+    # gives, chunk by chunk, exactly the outputs of the same steps run directly.
+    L = _lib()
+    w = W.WORKLOADS["768x1408"]
+    dev = torch.device("cuda")
+    chunks = [W.gen_layers(w, w.kv_len + i, w.q_layers) for i in range(5)]
+    prefill = [W.gen_layers(w, p, 1, "kv") for p in range(w.kv_len)]
+
+    def fresh_layer():
+        layer = L.LcsaLayer(w.heads, w.grid_h, w.grid_w, w.q_layers, w.kv_len, w.topk, device=dev)
+        for _, k, v in prefill:
+            layer.append(k.to(dev), v.to(dev))
+        return layer
+
+    direct = fresh_layer()
+    ref = []
+    for q, k, v in chunks:
+        out = torch.empty_like(q, device=dev)
+        direct.step(q.to(dev), k.to(dev), v.to(dev), out)
+        ref.append(out.cpu())
+    streamed = fresh_layer()
+    hs = L.HostStream(streamed, chunks[0][0].shape, dev)
+    pinned = [[t.pin_memory() for t in c] for c in chunks]
+    outs = [torch.empty_like(chunks[0][0]).pin_memory() for _ in chunks]
+    for (q, k, v), o in zip(pinned, outs):
+        hs.submit(q, k, v, o)
+    hs.drain_into(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert direct.status.item() == 0 and streamed.status.item() == 0
+    for o, r in zip(outs, ref):
+        assert torch.equal(o, r)
+
+
 # ------------------------------------------------------------------ edge cases
 
 def _tiny_setup(topk=8, heads=None):
