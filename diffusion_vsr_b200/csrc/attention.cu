@@ -265,6 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // copies.
         int g = 0, act = 0, r = 0;  // tiles, non-empty rows and rows so far
         bool ok = true;
+        // Launched as a programmatic dependent of the draft mask: its kept lists
+        // (and the ring the append before it wrote) are read only from here on.
+        grid_dep_wait();
         int cnt_next, idx_next;  // the next row's kept list, loaded one row ahead
         fetch_row(a, blockIdx.x, lane, cnt_next, idx_next);
         for (int unit = blockIdx.x; unit < a.n_units; unit += gridDim.x, ++r) {
@@ -636,7 +639,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                             const CUtensorMap &tm_o, const AttnArgs &a, void *out, cudaStream_t stream) {
+                             const CUtensorMap &tm_o, const AttnArgs &a, bool pdl, void *out,
+                             cudaStream_t stream) {
     const size_t smem = sizeof(AttnSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -645,8 +649,8 @@ cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, c
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const int grid = a.n_units < sms ? a.n_units : sms;
-    attention_kernel<<<grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, tm_o, a, static_cast<uint16_t *>(out));
-    return cudaGetLastError();
+    return launch_kernel(attention_kernel, dim3(grid), dim3(kThreads), smem, stream, pdl, tm_q, tm_k, tm_v, tm_o, a,
+                         static_cast<uint16_t *>(out));
 }
 
 }  // namespace lcsa

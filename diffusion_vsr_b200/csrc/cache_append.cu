@@ -14,6 +14,7 @@
 // are reduced in shared memory in a fixed order (deterministic).
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace lcsa {
 namespace {
@@ -21,6 +22,9 @@ namespace {
 constexpr int kThreads = 256;
 
 __global__ void __launch_bounds__(kThreads) cache_append_kernel(const AppendArgs a) {
+    // a draft mask launched as a programmatic dependent may start its q-mean
+    // phase now; it waits for this grid before reading the ring
+    grid_dep_launch();
     __shared__ float red[16][kHeadDim + 4];
     const int tid = threadIdx.x;
     const int chunk = tid & 15;  // dims [8*chunk, 8*chunk+8)

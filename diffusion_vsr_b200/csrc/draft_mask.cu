@@ -96,8 +96,9 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
     const int h = unit / (a.nblk * a.q_layers);
     const int qby = qb / a.grid_w;
     const int qbx = qb - qby * a.grid_w;
+    grid_dep_launch();  // the attention may start its set-up; it waits for this grid's lists
 
-    // ---- 1. block mean of q
+    // ---- 1. block mean of q (input of the caller: not written by the preceding kernel)
     {
         const size_t frame = static_cast<size_t>(h) * a.tq + ql * 2;
         const int half = lane >> 4, d8 = lane & 15;  // token parity, dims [8 d8, 8 d8 + 8)
@@ -156,6 +157,9 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
         if (a.qmean) a.qmean[static_cast<size_t>(unit) * kHeadDim + tid] = m;
     }
     __syncthreads();  // q mean and the -inf prefill are visible to every thread
+    // Launched as a programmatic dependent of the cache append: its key means
+    // are read only from here on (returns at once otherwise).
+    grid_dep_wait();
 
     // ---- 2. scores of the allowed candidates: warp w takes candidates
     //         64i + 8w ... 64i + 8w + 7; lane l reads dims [4l, 4l + 4) of each
@@ -314,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
 
 }  // namespace
 
-cudaError_t launch_draft(const DraftArgs &a, cudaStream_t stream) {
+cudaError_t launch_draft(const DraftArgs &a, bool pdl, cudaStream_t stream) {
     const int rows = a.heads * a.q_layers * a.nblk;
     const size_t smem = 4 * static_cast<size_t>(a.cand_cap);
     if (smem > 48 * 1024 - sizeof(DraftSmem)) {
@@ -322,8 +326,7 @@ cudaError_t launch_draft(const DraftArgs &a, cudaStream_t stream) {
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
-    draft_kernel<<<rows, kThreads, smem, stream>>>(a);
-    return cudaGetLastError();
+    return launch_kernel(draft_kernel, dim3(rows), dim3(kThreads), smem, stream, pdl, a);
 }
 
 }  // namespace lcsa

@@ -4,8 +4,28 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <utility>
 
 namespace lcsa {
+
+// Launch of `kernel` on `stream`, optionally as a programmatic dependent of the
+// stream's preceding kernel (it may start before that kernel completes and
+// waits for it with griddepcontrol.wait where it reads its results).
+template <typename... Params, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          bool pdl, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 constexpr int kBlockTokens = 128;
 constexpr int kHeadDim = 128;
@@ -37,7 +57,7 @@ struct AttnArgs {
 inline uint64_t div_magic_host(uint32_t d) { return ((1ull << 32) + d - 1) / d; }
 
 cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                             const CUtensorMap &tm_o, const AttnArgs &a, void *out, cudaStream_t stream);
+                             const CUtensorMap &tm_o, const AttnArgs &a, bool pdl, void *out, cudaStream_t stream);
 
 // Draft mask: q block means, scores over allowed candidates, top-k.
 struct DraftArgs {
@@ -55,7 +75,7 @@ struct DraftArgs {
     int32_t *status;
 };
 
-cudaError_t launch_draft(const DraftArgs &a, cudaStream_t stream);
+cudaError_t launch_draft(const DraftArgs &a, bool pdl, cudaStream_t stream);
 
 // Cache append: token layout -> block layout ring slots + k block means.
 struct AppendArgs {

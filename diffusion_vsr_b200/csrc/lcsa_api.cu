@@ -213,7 +213,8 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
     a.scores = scores_opt;
     a.qmean = qmean_opt;
     a.status = d_status;
-    if (lcsa::launch_draft(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LCSA_ERR_CUDA;
+    if (lcsa::launch_draft(a, (p->flags & LCSA_FLAG_PDL) != 0, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return LCSA_ERR_CUDA;
     return LCSA_OK;
 }
 
@@ -263,7 +264,8 @@ int lcsa_attention(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache 
     a.m_nq = lcsa::div_magic_host(static_cast<uint32_t>(nq));
     a.m_nblk = lcsa::div_magic_host(static_cast<uint32_t>(nblk));
     a.m_gw = lcsa::div_magic_host(static_cast<uint32_t>(p->grid_w));
-    if (lcsa::launch_attention(tq, tk, tv, to, a, out_tok, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (lcsa::launch_attention(tq, tk, tv, to, a, (p->flags & LCSA_FLAG_PDL) != 0, out_tok,
+                               static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LCSA_ERR_CUDA;
     return LCSA_OK;
 }

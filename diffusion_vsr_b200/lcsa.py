@@ -24,6 +24,7 @@ LCSA_ERR_CUDA = 3
 LCSA_ERR_TIMEOUT = 4
 LCSA_ERR_BAD_INDEX = 8
 LCSA_FLAG_FORCE_TIMEOUT = 1
+LCSA_FLAG_PDL = 2
 LCSA_MAX_CANDIDATES = 4096
 
 EXPORTED_SYMBOLS = ("lcsa_cache_append", "lcsa_draft_mask", "lcsa_attention", "lcsa_status_string",
@@ -180,6 +181,10 @@ class LcsaLayer:
     def __init__(self, heads: int, grid_h: int, grid_w: int, q_layers: int, kv_len: int, topk: int,
                  local_range: int = 11, local_mode: int = 0, device="cuda"):
         self.params = make_params(heads, grid_h, grid_w, q_layers, topk, local_range, local_mode)
+        # step(): the draft follows the append and the attention the draft, neither of
+        # which writes q or the output, so both may launch as programmatic dependents
+        self.params_chained = make_params(heads, grid_h, grid_w, q_layers, topk, local_range, local_mode,
+                                          flags=LCSA_FLAG_PDL)
         self.cache = KVCache.allocate(kv_len + q_layers, heads, grid_h, grid_w, device)
         nq = q_layers * grid_h * grid_w
         self.kept_idx = torch.empty((heads, nq, topk), dtype=torch.int32, device=device)
@@ -192,8 +197,8 @@ class LcsaLayer:
     def step(self, q_tok: torch.Tensor, k_tok: torch.Tensor, v_tok: torch.Tensor, out_tok: torch.Tensor,
              lse: Optional[torch.Tensor] = None) -> None:
         lcsa_cache_append(self.cache, k_tok, v_tok, d_status=self.status)
-        lcsa_draft_mask(self.params, q_tok, self.cache, self.kept_idx, self.kept_cnt, d_status=self.status)
-        lcsa_attention(self.params, q_tok, self.cache, self.kept_idx, self.kept_cnt, out_tok, lse,
+        lcsa_draft_mask(self.params_chained, q_tok, self.cache, self.kept_idx, self.kept_cnt, d_status=self.status)
+        lcsa_attention(self.params_chained, q_tok, self.cache, self.kept_idx, self.kept_cnt, out_tok, lse,
                        d_status=self.status)
 
 

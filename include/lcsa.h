@@ -55,6 +55,18 @@ enum lcsa_status {
 /* lcsa_params.flags */
 #define LCSA_FLAG_FORCE_TIMEOUT 1 /* test hook: the first consumer wait of
                                      lcsa_attention gives up at once */
+#define LCSA_FLAG_PDL 2           /* lcsa_draft_mask / lcsa_attention: launch as a
+                                     programmatic dependent of the kernel that
+                                     precedes it in the stream, so that it starts
+                                     while that kernel finishes.  The call waits
+                                     for that kernel (griddepcontrol.wait) before
+                                     reading the ring, the key means or the kept
+                                     lists, but reads q_tok before the wait: set it
+                                     only when the preceding kernel does not write
+                                     q_tok (nor, for lcsa_attention, out_tok or
+                                     lse_opt), e.g. when it is the cache append of
+                                     the same chunk (before the draft) or the draft
+                                     (before the attention). */
 
 #define LCSA_HEAD_DIM 128
 #define LCSA_BLOCK_TOKENS 128

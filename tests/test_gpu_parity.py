@@ -152,6 +152,39 @@ def test_deterministic_byte_identical():
     assert np.array_equal(a.out_pipeline, b.out_pipeline)
 
 
+def test_programmatic_dependent_launch_matches_plain_launches():
+    # LcsaLayer.step launches the draft and the attention as programmatic
+    # dependents (they start before the previous kernel completes and wait for
+    # its results in-kernel); over a stream with eviction the outputs and kept
+    # lists equal those of plain launches bit for bit.
+    L = _lib()
+    w = W.WORKLOADS["768x1408"]
+    dev = torch.device("cuda")
+    chunks = [[t.to(dev) for t in W.gen_layers(w, w.kv_len + i, w.q_layers)] for i in range(6)]
+    prefill = [[t.to(dev) for t in W.gen_layers(w, p, 1, "kv")[1:]] for p in range(w.kv_len)]
+    runs = []
+    for chained in (True, False):
+        layer = L.LcsaLayer(w.heads, w.grid_h, w.grid_w, w.q_layers, w.kv_len, w.topk, device=dev)
+        for k, v in prefill:
+            layer.append(k, v)
+        outs = []
+        for q, k, v in chunks:
+            out = torch.empty_like(q)
+            if chained:
+                layer.step(q, k, v, out)
+            else:
+                L.lcsa_cache_append(layer.cache, k, v, d_status=layer.status)
+                L.lcsa_draft_mask(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, d_status=layer.status)
+                L.lcsa_attention(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, out,
+                                 d_status=layer.status)
+            outs.append((out, layer.kept_idx.clone(), layer.kept_cnt.clone()))
+        torch.cuda.synchronize()
+        assert layer.status.item() == 0
+        runs.append(outs)
+    for (o1, k1, c1), (o2, k2, c2) in zip(*runs):
+        assert torch.equal(k1, k2) and torch.equal(c1, c2) and torch.equal(o1, o2)
+
+
 def test_host_stream_matches_direct_steps():
     # Overlapped host streaming (copy in / compute / copy out on three streams)
     # gives, chunk by chunk, exactly the outputs of the same steps run directly.
