@@ -131,3 +131,21 @@ def test_bench_takes_max_over_two_gloo_ranks():
     for rank, got, agg in out:
         assert got == 5.0
         assert abs(agg - 2 * 1e12 / 5e-3 / 1e12) < 1e-9
+
+
+def test_reference_arm_prints_one_json_line():
+    # `bench.py --impl reference` times the oracle (the pages ship no runnable
+    # reference) and prints one JSON line with the contract's keys.
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--steps", "2", "--warmup", "1"], capture_output=True, text=True, timeout=600, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
