@@ -240,7 +240,7 @@ def run_lcsa(args, rank: int, world: int, local_rank: int):
     value = aggregate_tflops(world, step_flops, ms_step)
 
     pk = peaks()
-    attn_ms = statistics.mean(t_attn)
+    attn_ms = statistics.mean(t_attn)  # the roofline uses the average launch time
     attn_tflops = step_flops / (attn_ms * 1e-3) / 1e12
     H, Nq, nblk = w.heads, w.n_query_blocks, w.blocks_per_layer
     q_bytes = H * Nq * 128 * 128 * 2
@@ -289,6 +289,9 @@ def run_lcsa(args, rank: int, world: int, local_rank: int):
         },
         "kernels": {
             "attention_ms": round(attn_ms, 5),
+            "attention_median_ms": round(statistics.median(t_attn), 5),
+            "draft_median_ms": round(statistics.median(t_draft), 5),
+            "cache_append_median_ms": round(statistics.median(t_append), 5),
             "draft_ms": round(draft_ms, 5),
             "draft_gbs": round(draft_bytes / (draft_ms * 1e-3) / 1e9, 1),
             "cache_append_ms": round(append_ms, 5),

@@ -10,7 +10,8 @@
 // blockIdx.x, blockIdx.x + gridDim.x, ... (head-major, so the CTAs running at
 // the same time share the key/value tiles of one or two heads in L2).
 // 384 threads, warp-specialised:
-//   warp 0         producer: validates each row's kept list (whole warp), then
+//   warp 0         producer: validates each row's kept list (whole warp; the
+//                  next row's list is loaded one row ahead), then
 //                  lane 0 issues the TMA copies — the Q tile straight from
 //                  token layout (rank-4 box of 2 x 8 x 8 tokens x 64 dims, so
 //                  the window partition costs nothing) into one of two Q
@@ -35,6 +36,9 @@
 //                  bf16 output tile in the row's Q buffer and writes it with one
 //                  TMA store into token layout (the reverse partition).
 // TMEM (512 columns): S_w at 128*w, O_w at 256 + 128*w.
+// Launched as a programmatic dependent of the draft mask (LCSA_FLAG_PDL), the
+// set-up overlaps the draft's tail and the producer waits for it before it
+// reads any kept list.
 // Every wait is bounded; on expiry the CTA drains its copies and MMAs, frees
 // TMEM and reports LCSA_ERR_TIMEOUT.
 
