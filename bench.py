@@ -187,10 +187,11 @@ def run_lcsa(args, rank: int, world: int, local_rank: int):
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
-        # the library's streaming step: append, then draft and attention each
-        # launched as a programmatic dependent of the kernel before it
+        # the library's streaming step, chained: the append runs in the SMs the
+        # previous step's attention leaves idle, the draft and the attention each
+        # start as the kernel before them finishes (programmatic dependent launch)
         q, k, v = chunks[i % n_bufs]
-        layer.step(q, k, v, out)
+        layer.step(q, k, v, out, overlap_previous=True)
 
     def step_split(i, ev):
         # the same three calls without programmatic dependence, with events between
@@ -270,10 +271,12 @@ def run_lcsa(args, rank: int, world: int, local_rank: int):
             "kv_len_layers": w.kv_len, "local_range": w.local_range, "topk": w.topk,
             "kept_tiles_per_chunk": kept_tiles, "tflop_per_chunk": round(step_flops / 1e12, 5),
             "l2": f"inputs larger than L2: {n_bufs} distinct chunk buffers rotated, ring "
-                  f"{w.capacity * H * nblk * 128 * 128 * 2 * 2 / 1e6:.0f} MB",
+                  f"{(layer.cache.k.numel() + layer.cache.v.numel()) * 2 / 1e6:.0f} MB "
+                  f"({layer.cache.desc.capacity} slots, {w.capacity} resident)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "launch": "append, then draft and attention each as a programmatic dependent of the kernel "
-                      "before it (LCSA_FLAG_PDL); per-kernel times from a separate pass without it",
+            "launch": "append, draft and attention each as a programmatic dependent of the kernel before "
+                      "it (LCSA_FLAG_PDL; the append writes a spare ring slot and overlaps the previous "
+                      "step's attention); per-kernel times from a separate pass of plain launches",
         },
         "roofline": {
             "kernel": "lcsa_attention (tcgen05 block-sparse attention)",

@@ -255,6 +255,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // Launched as a programmatic dependent of the draft mask, the set-up above
+    // overlapped its tail; its kept lists (and the ring the append before it
+    // wrote) are read only from here on.
+    grid_dep_wait();
+    // The next step's cache append may be launched as a programmatic dependent
+    // (its blocks take the SMs this grid's CTAs leave; it writes a spare ring
+    // slot).  Signalled only now: past the wait above, the previous step's
+    // kernels, which read that slot, have completed.
+    grid_dep_launch();
 
     // Copies issued by the producer (global counters), for the error-path drain.
     int k_issued = 0, v_issued = 0, q_issued = 0;
@@ -269,9 +278,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // copies.
         int g = 0, act = 0, r = 0;  // tiles, non-empty rows and rows so far
         bool ok = true;
-        // Launched as a programmatic dependent of the draft mask: its kept lists
-        // (and the ring the append before it wrote) are read only from here on.
-        grid_dep_wait();
         int cnt_next, idx_next;  // the next row's kept list, loaded one row ahead
         fetch_row(a, blockIdx.x, lane, cnt_next, idx_next);
         for (int unit = blockIdx.x; unit < a.n_units; unit += gridDim.x, ++r) {

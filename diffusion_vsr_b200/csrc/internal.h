@@ -88,6 +88,6 @@ struct AppendArgs {
     int32_t slots[kMaxAppendLayers];
 };
 
-cudaError_t launch_cache_append(const AppendArgs &a, cudaStream_t stream);
+cudaError_t launch_cache_append(const AppendArgs &a, bool pdl, cudaStream_t stream);
 
 }  // namespace lcsa

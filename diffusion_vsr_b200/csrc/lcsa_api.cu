@@ -49,11 +49,14 @@ int check_device() {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+int window_of(const lcsa_kv_cache *c) { return c->window > 0 ? c->window : c->capacity; }
+
 int check_cache(const lcsa_kv_cache *c) {
     if (!c || !c->k || !c->v || !c->kmean) return LCSA_ERR_INVALID_ARG;
     if (!aligned16(c->k) || !aligned16(c->v) || !aligned16(c->kmean)) return LCSA_ERR_INVALID_ARG;
     if (c->heads < 1 || c->grid_h < 1 || c->grid_w < 1 || c->capacity < 1) return LCSA_ERR_INVALID_ARG;
-    if (c->count < 0 || c->count > c->capacity || c->oldest < 0 || c->oldest >= c->capacity)
+    if (c->window < 0 || c->window > c->capacity) return LCSA_ERR_INVALID_ARG;
+    if (c->count < 0 || c->count > window_of(c) || c->oldest < 0 || c->oldest >= c->capacity)
         return LCSA_ERR_INVALID_ARG;
     // every token row index of the ring must fit a signed 32-bit TMA coordinate
     const int64_t rows = static_cast<int64_t>(c->capacity) * c->heads * c->grid_h * c->grid_w * kBlockTokens;
@@ -141,13 +144,17 @@ const char *lcsa_status_string(int code) {
     }
 }
 
-int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok, int32_t n_layers,
+int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok, int32_t n_layers, int32_t flags,
                       int32_t *d_status, void *stream) {
     (void)d_status;  // the append kernel has no device-side failure mode
     int rc = check_cache(cache);
     if (rc != LCSA_OK) return rc;
     if (!k_tok || !v_tok || !aligned16(k_tok) || !aligned16(v_tok)) return LCSA_ERR_INVALID_ARG;
-    if (n_layers < 1 || n_layers > cache->capacity || n_layers > lcsa::kMaxAppendLayers) return LCSA_ERR_INVALID_ARG;
+    const int window = window_of(cache);
+    if (n_layers < 1 || n_layers > window || n_layers > lcsa::kMaxAppendLayers) return LCSA_ERR_INVALID_ARG;
+    const bool pdl = (flags & LCSA_FLAG_PDL) != 0;
+    // overlapping the previous step is safe only while the new layers go to spare slots
+    if (pdl && n_layers > cache->capacity - window) return LCSA_ERR_INVALID_ARG;
     if ((rc = check_device()) != LCSA_OK) return rc;
 
     lcsa::AppendArgs a{};
@@ -165,15 +172,14 @@ int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok
     a.n_layers = n_layers;
     int oldest = cache->oldest, count = cache->count;
     for (int i = 0; i < n_layers; ++i) {
-        if (count < cache->capacity) {
-            a.slots[i] = (oldest + count) % cache->capacity;
+        a.slots[i] = (oldest + count) % cache->capacity;  // the slot after the newest layer
+        if (count < window) {
             ++count;
-        } else {  // ring full: the oldest layer is dropped and its slot reused
-            a.slots[i] = oldest;
+        } else {  // window full: the oldest layer is dropped
             oldest = (oldest + 1) % cache->capacity;
         }
     }
-    if (lcsa::launch_cache_append(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LCSA_ERR_CUDA;
+    if (lcsa::launch_cache_append(a, pdl, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LCSA_ERR_CUDA;
     cache->oldest = oldest;
     cache->count = count;
     return LCSA_OK;

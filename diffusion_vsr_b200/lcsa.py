@@ -41,7 +41,8 @@ class lcsa_params(ctypes.Structure):
 class lcsa_kv_cache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("kmean", ctypes.c_void_p),
                 ("capacity", ctypes.c_int32), ("oldest", ctypes.c_int32), ("count", ctypes.c_int32),
-                ("heads", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32)]
+                ("heads", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+                ("window", ctypes.c_int32)]
 
 
 class LcsaError(RuntimeError):
@@ -65,7 +66,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     P = ctypes.POINTER
     vp = ctypes.c_void_p
-    lib.lcsa_cache_append.argtypes = [P(lcsa_kv_cache), vp, vp, ctypes.c_int32, vp, vp]
+    lib.lcsa_cache_append.argtypes = [P(lcsa_kv_cache), vp, vp, ctypes.c_int32, ctypes.c_int32, vp, vp]
     lib.lcsa_cache_append.restype = ctypes.c_int
     lib.lcsa_draft_mask.argtypes = [P(lcsa_params), vp, P(lcsa_kv_cache), vp, vp, vp, vp, vp, vp]
     lib.lcsa_draft_mask.restype = ctypes.c_int
@@ -118,12 +119,15 @@ class KVCache:
     desc: lcsa_kv_cache
 
     @classmethod
-    def allocate(cls, capacity: int, heads: int, grid_h: int, grid_w: int, device="cuda") -> "KVCache":
+    def allocate(cls, capacity: int, heads: int, grid_h: int, grid_w: int, device="cuda",
+                 window: int = 0) -> "KVCache":
+        """``capacity`` slots of which at most ``window`` layers are resident (0: all)."""
         nblk = grid_h * grid_w
         k = torch.empty((capacity, heads, nblk, 128, 128), dtype=torch.bfloat16, device=device)
         v = torch.empty_like(k)
         km = torch.empty((capacity, heads, nblk, 128), dtype=torch.float32, device=device)
-        desc = lcsa_kv_cache(k.data_ptr(), v.data_ptr(), km.data_ptr(), capacity, 0, 0, heads, grid_h, grid_w)
+        desc = lcsa_kv_cache(k.data_ptr(), v.data_ptr(), km.data_ptr(), capacity, 0, 0, heads, grid_h, grid_w,
+                             window)
         return cls(k, v, km, desc)
 
     @property
@@ -143,10 +147,10 @@ class KVCache:
 
 
 def lcsa_cache_append(cache: KVCache, k_tok: torch.Tensor, v_tok: torch.Tensor, n_layers: Optional[int] = None,
-                      d_status: Optional[torch.Tensor] = None, stream=None) -> None:
+                      d_status: Optional[torch.Tensor] = None, stream=None, flags: int = 0) -> None:
     if n_layers is None:
         n_layers = k_tok.shape[1] // 2
-    rc = load_library().lcsa_cache_append(ctypes.byref(cache.desc), _ptr(k_tok), _ptr(v_tok), n_layers,
+    rc = load_library().lcsa_cache_append(ctypes.byref(cache.desc), _ptr(k_tok), _ptr(v_tok), n_layers, flags,
                                           _ptr(d_status), _stream(stream))
     _check("lcsa_cache_append", rc)
 
@@ -185,7 +189,10 @@ class LcsaLayer:
         # which writes q or the output, so both may launch as programmatic dependents
         self.params_chained = make_params(heads, grid_h, grid_w, q_layers, topk, local_range, local_mode,
                                           flags=LCSA_FLAG_PDL)
-        self.cache = KVCache.allocate(kv_len + q_layers, heads, grid_h, grid_w, device)
+        # kv_len + q_layers resident layers plus q_layers spare slots: a step's append
+        # never overwrites a layer the previous step reads (see step(overlap_previous))
+        self.cache = KVCache.allocate(kv_len + 2 * q_layers, heads, grid_h, grid_w, device,
+                                      window=kv_len + q_layers)
         nq = q_layers * grid_h * grid_w
         self.kept_idx = torch.empty((heads, nq, topk), dtype=torch.int32, device=device)
         self.kept_cnt = torch.empty((heads, nq), dtype=torch.int32, device=device)
@@ -195,8 +202,16 @@ class LcsaLayer:
         lcsa_cache_append(self.cache, k_tok, v_tok, d_status=self.status)
 
     def step(self, q_tok: torch.Tensor, k_tok: torch.Tensor, v_tok: torch.Tensor, out_tok: torch.Tensor,
-             lse: Optional[torch.Tensor] = None) -> None:
-        lcsa_cache_append(self.cache, k_tok, v_tok, d_status=self.status)
+             lse: Optional[torch.Tensor] = None, overlap_previous: bool = False) -> None:
+        """Append the chunk's k/v, build the draft mask, run the attention.
+
+        overlap_previous: the kernel before this call in the stream is the previous
+        step's attention (or anything else that writes neither k_tok nor v_tok);
+        the append is then launched as its programmatic dependent and runs in the
+        SMs that attention's last CTAs leave idle.
+        """
+        lcsa_cache_append(self.cache, k_tok, v_tok, d_status=self.status,
+                          flags=LCSA_FLAG_PDL if overlap_previous else 0)
         lcsa_draft_mask(self.params_chained, q_tok, self.cache, self.kept_idx, self.kept_cnt, d_status=self.status)
         lcsa_attention(self.params_chained, q_tok, self.cache, self.kept_idx, self.kept_cnt, out_tok, lse,
                        d_status=self.status)
@@ -247,7 +262,9 @@ class HostStream:
         self.compute.wait_event(self.in_ready[b])
         self.compute.wait_event(self.copied_out[b])
         with torch.cuda.stream(self.compute):
-            self.layer.step(q, k, v, self.outputs[b])
+            # the kernel before this step on the compute stream is the previous
+            # chunk's attention (or none): the append may overlap it
+            self.layer.step(q, k, v, self.outputs[b], overlap_previous=True)
         self.computed[b].record(self.compute)
         self.copy_out.wait_event(self.computed[b])
         with torch.cuda.stream(self.copy_out):

@@ -55,18 +55,24 @@ enum lcsa_status {
 /* lcsa_params.flags */
 #define LCSA_FLAG_FORCE_TIMEOUT 1 /* test hook: the first consumer wait of
                                      lcsa_attention gives up at once */
-#define LCSA_FLAG_PDL 2           /* lcsa_draft_mask / lcsa_attention: launch as a
-                                     programmatic dependent of the kernel that
-                                     precedes it in the stream, so that it starts
-                                     while that kernel finishes.  The call waits
-                                     for that kernel (griddepcontrol.wait) before
-                                     reading the ring, the key means or the kept
-                                     lists, but reads q_tok before the wait: set it
-                                     only when the preceding kernel does not write
-                                     q_tok (nor, for lcsa_attention, out_tok or
-                                     lse_opt), e.g. when it is the cache append of
-                                     the same chunk (before the draft) or the draft
-                                     (before the attention). */
+#define LCSA_FLAG_PDL 2           /* launch as a programmatic dependent of the
+                                     kernel that precedes the call in the stream,
+                                     so that it starts while that kernel finishes.
+                                     lcsa_draft_mask / lcsa_attention wait for that
+                                     kernel (griddepcontrol.wait) before reading
+                                     the ring, the key means or the kept lists, but
+                                     read q_tok before the wait: set the flag only
+                                     when the preceding kernel does not write q_tok
+                                     (nor, for lcsa_attention, out_tok or lse_opt),
+                                     e.g. when it is the cache append of the same
+                                     chunk (before the draft) or the draft (before
+                                     the attention).  lcsa_cache_append (flags
+                                     argument) writes the ring before the wait and
+                                     waits only at its end: set it only when the
+                                     preceding kernel writes neither k_tok nor v_tok
+                                     and the new layers fit the ring's spare slots
+                                     (n_layers <= capacity - window), e.g. when it
+                                     is the previous chunk's lcsa_attention. */
 
 #define LCSA_HEAD_DIM 128
 #define LCSA_BLOCK_TOKENS 128
@@ -91,17 +97,23 @@ typedef struct lcsa_params {
  *   k, v   bf16 [capacity][heads][grid_h*grid_w][128 tokens][128]
  *   kmean  fp32 [capacity][heads][grid_h*grid_w][128]  (block means of k)
  * Slot of logical layer L: (oldest + L) % capacity.  `oldest` and `count`
- * are host-side state updated by lcsa_cache_append; start from 0, 0. */
+ * are host-side state updated by lcsa_cache_append; start from 0, 0.
+ * At most `window` layers are resident (kv_len + layers of one step); the
+ * slots beyond the window (capacity - window of them) are spares: a new layer
+ * goes into the slot after the newest one, so that it never overwrites a layer
+ * of the previous window (what lets an append overlap the previous step, see
+ * LCSA_FLAG_PDL). window = 0 means window = capacity (no spare slot). */
 typedef struct lcsa_kv_cache {
     void *k;
     void *v;
     float *kmean;
-    int32_t capacity; /* kv_len + layers of one step */
+    int32_t capacity; /* slots: window, plus spares */
     int32_t oldest;
-    int32_t count;
+    int32_t count;    /* resident layers, <= window */
     int32_t heads;
     int32_t grid_h;
     int32_t grid_w;
+    int32_t window;   /* 0 < window <= capacity, or 0 for capacity */
 } lcsa_kv_cache;
 
 /*
@@ -109,13 +121,15 @@ typedef struct lcsa_kv_cache {
  * (learn.html 2.3: the cache keeps the newest layers and drops the oldest).
  *   k_tok, v_tok: bf16 token layout [heads][2*n_layers][8*grid_h][8*grid_w][128].
  * Each layer is written in block layout (partition of learn.html 2.2) into
- * the next ring slot, together with its fp32 block means of k; when the
- * ring is full the oldest layer's slot is overwritten and `oldest` advances.
+ * the slot after the newest layer, together with its fp32 block means of k;
+ * when `window` layers are resident the oldest is dropped and `oldest`
+ * advances (without spare slots its slot is the one reused).
+ *   flags: 0 or LCSA_FLAG_PDL (see there).
  * Updates cache->oldest/count on the host when the copy is enqueued, so calls
  * on one cache must be serialised by the caller.  1 <= n_layers <= capacity.
  */
 int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok,
-                      int32_t n_layers, int32_t *d_status, void *stream);
+                      int32_t n_layers, int32_t flags, int32_t *d_status, void *stream);
 
 /*
  * lcsa_draft_mask - the draft mask of learn.html 2.2, one row per

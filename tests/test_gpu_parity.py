@@ -153,10 +153,11 @@ def test_deterministic_byte_identical():
 
 
 def test_programmatic_dependent_launch_matches_plain_launches():
-    # LcsaLayer.step launches the draft and the attention as programmatic
-    # dependents (they start before the previous kernel completes and wait for
-    # its results in-kernel); over a stream with eviction the outputs and kept
-    # lists equal those of plain launches bit for bit.
+    # LcsaLayer.step(overlap_previous=True) launches all three kernels as
+    # programmatic dependents (each starts before the previous kernel completes
+    # and waits for its results in-kernel; the append writes a spare ring slot
+    # while the previous step's attention still runs); over a stream with
+    # eviction the outputs and kept lists equal those of plain launches bit for bit.
     L = _lib()
     w = W.WORKLOADS["768x1408"]
     dev = torch.device("cuda")
@@ -171,7 +172,7 @@ def test_programmatic_dependent_launch_matches_plain_launches():
         for q, k, v in chunks:
             out = torch.empty_like(q)
             if chained:
-                layer.step(q, k, v, out)
+                layer.step(q, k, v, out, overlap_previous=True)
             else:
                 L.lcsa_cache_append(layer.cache, k, v, d_status=layer.status)
                 L.lcsa_draft_mask(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, d_status=layer.status)

@@ -56,13 +56,29 @@ def _fake_cache(**kw):
 
 def test_cache_append_rejects_bad_arguments_without_touching_the_gpu(lib):
     c = _fake_cache()
-    assert lib.lcsa_cache_append(None, 0x40000, 0x50000, 1, None, None) == L.LCSA_ERR_INVALID_ARG
-    assert lib.lcsa_cache_append(ctypes.byref(c), None, 0x50000, 1, None, None) == L.LCSA_ERR_INVALID_ARG
-    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40008, 0x50000, 1, None, None) == L.LCSA_ERR_INVALID_ARG
-    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 5, None, None) == L.LCSA_ERR_INVALID_ARG
-    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(None, 0x40000, 0x50000, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), None, 0x50000, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40008, 0x50000, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 5, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 0, 0, None, None) == L.LCSA_ERR_INVALID_ARG
     bad = _fake_cache(count=5)
-    assert lib.lcsa_cache_append(ctypes.byref(bad), 0x40000, 0x50000, 1, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(bad), 0x40000, 0x50000, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+
+
+def test_cache_window_and_overlap_rules(lib):
+    k, v = 0x40000, 0x50000
+    # at most `window` layers resident, window <= capacity
+    wide = _fake_cache(capacity=5, window=6, count=4)
+    assert lib.lcsa_cache_append(ctypes.byref(wide), k, v, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    over = _fake_cache(capacity=5, window=4, count=5)
+    assert lib.lcsa_cache_append(ctypes.byref(over), k, v, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    # an append overlapping the previous step must fit the spare slots (5 - 4 = 1 here)
+    ok = _fake_cache(capacity=5, window=4, count=4)
+    assert lib.lcsa_cache_append(ctypes.byref(ok), k, v, 2, L.LCSA_FLAG_PDL, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(ok), k, v, 1, L.LCSA_FLAG_PDL, None, None) != L.LCSA_ERR_INVALID_ARG
+    no_spare = _fake_cache(capacity=4, window=0, count=4)
+    assert lib.lcsa_cache_append(ctypes.byref(no_spare), k, v, 1, L.LCSA_FLAG_PDL, None, None) == \
+        L.LCSA_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("field,value", [("head_dim", 64), ("topk", 0), ("local_range", 4), ("local_mode", 2),
