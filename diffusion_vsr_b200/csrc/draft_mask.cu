@@ -20,13 +20,15 @@
 //     key mean is one coalesced warp load, dotted with the q mean in fp32
 //     (per-lane partial products, then a fixed reduce-scatter butterfly);
 //  3. exact top-k: scores become 32-bit keys whose unsigned order is the
-//     descending score order; a 4-pass radix select (8 bits per pass, block
-//     histogram in shared memory, one atomic per distinct bin and warp) finds
-//     the k-th key T; warp 0 writes every
+//     descending score order; a radix select of up to 4 passes (8 bits per
+//     pass, block histogram in shared memory, one atomic per distinct bin and
+//     warp; it stops after the pass whose bin holding the k-th key is kept
+//     whole) finds the k-th key T; warp 0 writes every
 //     key < T plus the first (lowest-index) keys equal to T, in ascending key
 //     index, by a ballot compaction.
 
 #include <cfloat>
+#include <climits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -67,9 +69,19 @@ __device__ __forceinline__ uint32_t desc_key(float score) {
 
 // Exact n / d for 0 <= n, d < 2^16 (d >= 1) with m = ceil(2^32 / d): the
 // rounding excess of n m / 2^32 over n / d is below n / 2^32 < 1 / d.
-__device__ __forceinline__ uint64_t div_magic(uint32_t d) { return ((1ull << 32) + d - 1) / d; }
+// ceil(2^32 / d) = floor((2^32 - 1) / d) + 1 for every d >= 1, a 32-bit division.
+__device__ __forceinline__ uint64_t div_magic(uint32_t d) { return static_cast<uint64_t>(0xFFFFFFFFu / d) + 1u; }
 __device__ __forceinline__ int div_by(int n, uint64_t m) {
     return static_cast<int>((static_cast<uint64_t>(static_cast<uint32_t>(n)) * m) >> 32);
+}
+
+// lo += low bf16 of w, hi += high bf16 of w: mixed-precision fp32 adds (the
+// bf16 operand widens exactly, one rounding, as a plain fp32 add would do).
+__device__ __forceinline__ void add_bf16x2(float &lo, float &hi, uint32_t w) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(w));
 }
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
@@ -82,7 +94,7 @@ struct DraftSmem {
     __align__(16) float part[kWarps][kHeadDim];  // per-warp partial sums of q
     __align__(16) float mq[kHeadDim];
     uint32_t hist[256];
-    uint32_t digit, below;
+    uint32_t digit, below, whole;
 };
 
 __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
@@ -91,10 +103,11 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int unit = blockIdx.x;  // (head, query layer, query block) row
-    const int qb = unit % a.nblk;
-    const int ql = (unit / a.nblk) % a.q_layers;
-    const int h = unit / (a.nblk * a.q_layers);
-    const int qby = qb / a.grid_w;
+    const int h = div_by(unit, a.m_nq);
+    const int qi = unit - h * a.nblk * a.q_layers;
+    const int ql = div_by(qi, a.m_nblk);
+    const int qb = qi - ql * a.nblk;
+    const int qby = div_by(qb, a.m_gw);
     const int qbx = qb - qby * a.grid_w;
     grid_dep_launch();  // the attention may start its set-up; it waits for this grid's lists
 
@@ -117,10 +130,7 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
         for (int i = 0; i < 8; ++i) {
             const uint32_t w4[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                acc[2 * e] += __uint_as_float(w4[e] << 16);
-                acc[2 * e + 1] += __uint_as_float(w4[e] & 0xFFFF0000u);
-            }
+            for (int e = 0; e < 4; ++e) add_bf16x2(acc[2 * e], acc[2 * e + 1], w4[e]);
         }
         // even tokens (lanes 0-15) + odd tokens (lanes 16-31)
 #pragma unroll
@@ -236,6 +246,7 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
     // ---- 3. exact top-k: radix select of the k-th smallest key
     const int k = min(a.topk, ncand);
     uint32_t prefix = 0, mask = 0, k_rem = static_cast<uint32_t>(k);
+    bool whole = false;
 #pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
@@ -272,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
                     if (run + cnt[e] >= k_rem) {
                         sm.digit = static_cast<uint32_t>(lane * 8 + e);
                         sm.below = run;
+                        sm.whole = run + cnt[e] == k_rem;  // every key of the bin is kept
                         break;
                     }
                     run += cnt[e];
@@ -282,10 +294,16 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
         k_rem -= sm.below;
         prefix |= sm.digit << shift;
         mask |= 255u << shift;
+        if (sm.whole) {  // the k-th key's bin is kept whole: no further digit is needed
+            prefix |= (1u << shift) - 1u;  // T = the largest key of the bin
+            whole = true;
+            break;
+        }
     }
     if (warp != 0) return;
     const uint32_t T = prefix;
-    const int k_eq = static_cast<int>(k_rem);  // keys equal to T that belong to the k smallest
+    // keys equal to T that belong to the k smallest (all of them when the bin is kept whole)
+    const int k_eq = whole ? INT_MAX : static_cast<int>(k_rem);
 
     // kept set in ascending key index
     int32_t *out = a.kept_idx + static_cast<size_t>(unit) * a.topk;

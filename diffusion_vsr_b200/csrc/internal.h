@@ -67,6 +67,7 @@ struct DraftArgs {
     int32_t capacity, oldest, count;
     int32_t local_range, local_mode, topk;
     int32_t cand_cap;      // most allowed candidates of a row, rounded up to 32
+    uint64_t m_nq, m_nblk, m_gw;  // multiply-high multipliers of q_layers*nblk, nblk, grid_w
     float scale;
     int32_t *kept_idx;
     int32_t *kept_cnt;
