@@ -9,8 +9,8 @@
 // contiguous 32 KB block.  The fp32 block means of k used by the draft mask
 // (section 2.2, avgpool_k) are produced in the same pass.
 //
-// 256-thread CTAs walk the (new layer, head, block) units grid-stride (at
-// most four CTAs per SM, so that the grid also fits the SMs a finishing
+// 256-thread CTAs walk the (new layer, head, block) units grid-stride (a
+// grid of at most two CTAs per SM, so that it also fits the SMs a finishing
 // kernel leaves free): 16 threads per 256-byte token row, 16-byte loads and
 // stores, 128 tokens of k and of v per unit; the k means are reduced in shared
 // memory in a fixed order (deterministic).
@@ -81,8 +81,11 @@ __global__ void __launch_bounds__(kThreads) cache_append_kernel(const AppendArgs
     }
     // Launched as a programmatic dependent of the previous step's attention (it
     // writes a spare slot that kernel does not read), this grid completes only
-    // after that kernel: whoever waits for this grid waits for both.
-    grid_dep_wait();
+    // after that kernel: whoever waits for this grid waits for both.  One CTA
+    // waiting is enough for that (a grid completes when its last CTA exits); the
+    // others exit at once and leave their SM slots to the kernels chained after
+    // this one.
+    if (blockIdx.x == 0) grid_dep_wait();
 }
 
 }  // namespace

@@ -19,6 +19,9 @@
 //     window row, then window column), eight per warp at a time: each 512-byte
 //     key mean is one coalesced warp load, dotted with the q mean in fp32
 //     (per-lane partial products, then a fixed reduce-scatter butterfly);
+//     chained after the chunk's cache append, the candidates of the older
+//     layers are scored while the append still runs, those of the chunk's own
+//     layers after it;
 //  3. exact top-k: scores become 32-bit keys whose unsigned order is the
 //     descending score order; a radix select of up to 4 passes (8 bits per
 //     pass, block histogram in shared memory, one atomic per distinct bin and
@@ -167,24 +170,21 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
         if (a.qmean) a.qmean[static_cast<size_t>(unit) * kHeadDim + tid] = m;
     }
     __syncthreads();  // q mean and the -inf prefill are visible to every thread
-    // Launched as a programmatic dependent of the cache append: its key means
-    // are read only from here on (returns at once otherwise).
-    grid_dep_wait();
 
-    // ---- 2. scores of the allowed candidates: warp w takes candidates
-    //         64i + 8w ... 64i + 8w + 7; lane l reads dims [4l, 4l + 4) of each
-    //         (one coalesced 512-byte row per load, 8 in flight), fp32
+    // ---- 2. scores of the allowed candidates in [c_begin, c_end): warp w takes
+    //         candidates c_begin + 64i + 8w ... + 7; lane l reads dims [4l, 4l + 4)
+    //         of each (one coalesced 512-byte row per load, 8 in flight), fp32
     //         products, then a fixed reduce-scatter butterfly.
-    {
+    const float4 qv = reinterpret_cast<const float4 *>(sm.mq)[lane];
+    auto score_range = [&](int c_begin, int c_end) {
         constexpr int kU = 8;
-        const float4 qv = reinterpret_cast<const float4 *>(sm.mq)[lane];
-        for (int c0 = warp * kU; c0 < ncand; c0 += kWarps * kU) {
+        for (int c0 = c_begin + warp * kU; c0 < c_end; c0 += kWarps * kU) {
             // lane u < kU locates candidate c0 + u (one division pair per lane),
             // then every lane loads its 16 bytes of each of the kU rows
             const float4 *row = nullptr;
             int jl = 0;
             if (lane < kU) {
-                const int c = min(c0 + lane, ncand - 1);
+                const int c = min(c0 + lane, c_end - 1);
                 const int layer = div_by(c, m_wsz);
                 const int rem = c - layer * wsz;
                 const int ry = div_by(rem, m_wx);
@@ -235,13 +235,23 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
             d1 += __shfl_xor_sync(kFull, d1, 1);
             const int u = lane >> 2;
             const int jl_u = __shfl_sync(kFull, jl, u);
-            if ((lane & 3) == 0 && c0 + u < ncand) {
+            if ((lane & 3) == 0 && c0 + u < c_end) {
                 const float score = d1 * a.scale;
                 keys[c0 + u] = desc_key(score);
                 if (srow) srow[jl_u] = score;
             }
         }
-    }
+    };
+    // Candidates of the layers resident before the chunk (logical layers below
+    // count - q_layers, written by earlier appends) are scored at once; those of
+    // the chunk's own layers only after the wait below.
+    const int c_split = min(ncand, max(a.count - a.q_layers, 0) * wsz);
+    score_range(0, c_split);
+    // Launched as a programmatic dependent of the cache append of the chunk:
+    // the key means of its layers are read only from here on (returns at once
+    // otherwise).
+    grid_dep_wait();
+    score_range(c_split, ncand);
 
     // ---- 3. exact top-k: radix select of the k-th smallest key
     const int k = min(a.topk, ncand);

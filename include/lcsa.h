@@ -60,13 +60,16 @@ enum lcsa_status {
                                      so that it starts while that kernel finishes.
                                      lcsa_draft_mask / lcsa_attention wait for that
                                      kernel (griddepcontrol.wait) before reading
-                                     the ring, the key means or the kept lists, but
-                                     read q_tok before the wait: set the flag only
-                                     when the preceding kernel does not write q_tok
+                                     the ring, the kept lists or the key means of
+                                     the newest q_layers layers, but read q_tok
+                                     (and the draft the key means of the older
+                                     layers) before the wait: set the flag only
+                                     when the preceding kernel writes none of these
                                      (nor, for lcsa_attention, out_tok or lse_opt),
                                      e.g. when it is the cache append of the same
-                                     chunk (before the draft) or the draft (before
-                                     the attention).  lcsa_cache_append (flags
+                                     chunk (before the draft: it writes only the
+                                     chunk's own, newest layers) or the draft
+                                     (before the attention).  lcsa_cache_append (flags
                                      argument) writes the ring before the wait and
                                      waits only at its end: set it only when the
                                      preceding kernel writes neither k_tok nor v_tok
