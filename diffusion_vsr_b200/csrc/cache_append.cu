@@ -9,95 +9,165 @@
 // contiguous 32 KB block.  The fp32 block means of k used by the draft mask
 // (section 2.2, avgpool_k) are produced in the same pass.
 //
-// 256-thread CTAs walk the (new layer, head, block) units grid-stride (a
-// grid of at most two CTAs per SM, so that it also fits the SMs a finishing
-// kernel leaves free): 16 threads per 256-byte token row, 16-byte loads and
-// stores, 128 tokens of k and of v per unit; the k means are reduced in shared
-// memory in a fixed order (deterministic).
+// A copy engine kernel: one 128-thread CTA per SM walks the (new layer, head,
+// block) units grid-stride.  For each unit one thread issues two TMA loads
+// (a (128 dims, 8, 8, 2 frames) box of k and of v lands in shared memory
+// already in block order: intra index (t, y, x) row-major) and, once the
+// threads have read the k tile for its mean, two 32 KB bulk stores into the
+// ring slot.  Two stages: the loads of the next unit are in flight while the
+// current one is reduced and stored.  The k mean of a dimension is the sum of
+// the 128 tokens in a fixed order (two halves of 64 tokens, then half 0 +
+// half 1), times 1/128: deterministic.  Few registers and one CTA per SM, so
+// that the grid fits the SMs a finishing kernel leaves free next to the CTAs
+// of the kernel chained after it.
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "../../include/lcsa.h"
 
 namespace lcsa {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
+constexpr int kStages = 2;
+constexpr uint32_t kTileBytes = kBlockTokens * kHeadDim * 2;  // 32 KB
 
-__global__ void __launch_bounds__(kThreads) cache_append_kernel(const AppendArgs a) {
-    // a draft mask launched as a programmatic dependent may start its q-mean
-    // phase now; it waits for this grid before reading the ring
+struct __align__(1024) AppendSmem {
+    uint16_t k[kStages][kBlockTokens * kHeadDim];
+    uint16_t v[kStages][kBlockTokens * kHeadDim];
+    float2 part[kStages][kHeadDim / 2];  // sums over tokens 64..127, per dimension pair
+    uint64_t full[kStages];
+    int abort_word;
+};
+
+__device__ __forceinline__ int mul_div(int n, uint64_t m) {
+    return static_cast<int>((static_cast<uint64_t>(static_cast<uint32_t>(n)) * m) >> 32);
+}
+
+struct Unit {
+    int li, h, b;
+};
+
+// unit = (layer within the chunk, head, block), block fastest
+__device__ __forceinline__ Unit unit_of(const AppendArgs &a, int u) {
+    Unit r;
+    const int hb = mul_div(u, a.m_nblk);
+    r.b = u - hb * a.nblk;
+    r.li = mul_div(hb, a.m_heads);
+    r.h = hb - r.li * a.heads;
+    return r;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    cache_append_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        const AppendArgs a) {
+    // a draft mask launched as a programmatic dependent may start now; it waits
+    // for this grid before it reads what this grid writes
     grid_dep_launch();
     // (a preceding kernel this grid depends on programmatically is waited for
-    // at the end: the k/v inputs are the caller's and the slot is a spare)
-    __shared__ float red[16][kHeadDim + 4];
+    // at the end: the k/v inputs are the caller's and the slots are spare)
+    extern __shared__ uint8_t smem_raw[];
+    AppendSmem &sm = *reinterpret_cast<AppendSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                      ~static_cast<uintptr_t>(1023));
     const int tid = threadIdx.x;
-    const int chunk = tid & 15;  // dims [8*chunk, 8*chunk+8)
-    const int sub = tid >> 4;    // token sub-group 0..15
-    const int tc = 2 * a.n_layers;  // frames of the chunk
     const int n_units = a.n_layers * a.heads * a.nblk;
-    // grid-stride over (layer, head, block) units: a grid of a few CTAs per SM
-    // fits into whatever SMs are free when it is launched
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-        int unit = u;
-        const int b = unit % a.nblk;
-        unit /= a.nblk;
-        const int h = unit % a.heads;
-        const int li = unit / a.heads;  // layer within the appended chunk
-        const int by = b / a.grid_w, bx = b - by * a.grid_w;
-        const int slot = a.slots[li];
+    const int n_mine = blockIdx.x < n_units ? (n_units - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
+    const int tc = 2 * a.n_layers;  // frames of the chunk
+    volatile int *abort_word = &sm.abort_word;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&sm.full[s]), 1);
+        sm.abort_word = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    __syncthreads();
 
-        const size_t dst_block = ((static_cast<size_t>(slot) * a.heads + h) * a.nblk + b) * kBlockTokens;
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-        for (int it = 0; it < 8; ++it) {
-            const int n = sub + 16 * it;  // token of the block, (t, y, x) row-major
-            const int t = n >> 6, y = (n >> 3) & 7, x = n & 7;
-            const size_t src = ((static_cast<size_t>(h) * tc + li * 2 + t) * a.tok_h + by * 8 + y) * a.tok_w + bx * 8 + x;
-            const size_t so = src * kHeadDim + chunk * 8;
-            const size_t dof = (dst_block + n) * kHeadDim + chunk * 8;
-            const uint4 kr = __ldg(reinterpret_cast<const uint4 *>(a.k_tok + so));
-            const uint4 vr = __ldg(reinterpret_cast<const uint4 *>(a.v_tok + so));
-            *reinterpret_cast<uint4 *>(a.k_cache + dof) = kr;
-            *reinterpret_cast<uint4 *>(a.v_cache + dof) = vr;
-            const uint32_t w[4] = {kr.x, kr.y, kr.z, kr.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                acc[2 * e] += __uint_as_float(w[e] << 16);
-                acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+    auto issue_load = [&](int i) {  // the i-th unit of this CTA into stage i % kStages
+        const Unit un = unit_of(a, static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x));
+        const int by = mul_div(un.b, a.m_gw), bx = un.b - by * a.grid_w;
+        const int s = i % kStages;
+        const uint32_t bar = smem_u32(&sm.full[s]);
+        mbar_arrive_expect_tx(bar, 2 * kTileBytes);
+        tma_load_4d(smem_u32(sm.k[s]), &tm_k, bar, 0, bx * 8, by * 8, un.h * tc + 2 * un.li);
+        tma_load_4d(smem_u32(sm.v[s]), &tm_v, bar, 0, bx * 8, by * 8, un.h * tc + 2 * un.li);
+    };
+    int issued = 0;  // loads issued (thread 0)
+    if (tid == 0) {
+        for (; issued < kStages && issued < n_mine; ++issued) issue_load(issued);
+    }
+
+    const int pr = tid & 63;   // dimensions 2 pr, 2 pr + 1
+    const int half = tid >> 6;  // tokens [64 half, 64 half + 64)
+    bool ok = true;
+    for (int i = 0; i < n_mine; ++i) {
+        const int s = i % kStages;
+        ok = mbar_wait(smem_u32(&sm.full[s]), (i / kStages) & 1, abort_word, a.timeout_ns);
+        if (!__syncthreads_and(ok)) {
+            ok = false;
+            break;
+        }
+        const Unit un = unit_of(a, static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x));
+        const size_t blk = (static_cast<size_t>(a.slots[un.li]) * a.heads + un.h) * a.nblk + un.b;
+        // k mean: this thread sums its 64 tokens of two dimensions
+        const uint32_t *kw = reinterpret_cast<const uint32_t *>(sm.k[s]) + half * 64 * (kHeadDim / 2) + pr;
+        float lo = 0.f, hi = 0.f;
+#pragma unroll 16
+        for (int n = 0; n < 64; ++n) add_bf16x2(lo, hi, kw[n * (kHeadDim / 2)]);
+        if (half == 1) sm.part[s][pr] = make_float2(lo, hi);
+        __syncthreads();  // every thread has read the k tile; the upper-half sums are visible
+        if (tid == 0) {
+            // the tiles go to the ring slot unchanged: two bulk stores
+            fence_proxy_async_smem();
+            bulk_store(a.k_cache + blk * kBlockTokens * kHeadDim, smem_u32(sm.k[s]), kTileBytes);
+            bulk_store(a.v_cache + blk * kBlockTokens * kHeadDim, smem_u32(sm.v[s]), kTileBytes);
+            bulk_commit_group();
+            if (issued < n_mine) {
+                // stage s is refilled once the stores above have read it
+                bulk_wait_group_read0();
+                issue_load(issued++);
             }
         }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) red[sub][chunk * 8 + e] = acc[e];
-        __syncthreads();
-        if (tid < kHeadDim) {
-            float s = 0.f;
-#pragma unroll
-            for (int g = 0; g < 16; ++g) s += red[g][tid];
-            a.kmean[((static_cast<size_t>(slot) * a.heads + h) * a.nblk + b) * kHeadDim + tid] = s * (1.0f / 128.0f);
+        if (half == 0) {
+            const float2 up = sm.part[s][pr];
+            reinterpret_cast<float2 *>(a.kmean + blk * kHeadDim)[pr] =
+                make_float2((lo + up.x) * (1.0f / 128.0f), (hi + up.y) * (1.0f / 128.0f));
         }
-        __syncthreads();  // red is reused by the next unit
+    }
+    if (tid == 0) {
+        if (!ok) {
+            // a wait gave up: the loads still in flight (among the last kStages
+            // issued; a consumed one passes at once) land before the CTA exits
+            for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+                mbar_wait_drain(smem_u32(&sm.full[i % kStages]), (i / kStages) & 1, a.timeout_ns);
+            if (a.status) atomicOr(a.status, LCSA_ERR_TIMEOUT);
+        }
+        bulk_wait_group0();  // the stores have completed before the shared memory is released
     }
     // Launched as a programmatic dependent of the previous step's attention (it
-    // writes a spare slot that kernel does not read), this grid completes only
+    // writes spare slots that kernel does not read), this grid completes only
     // after that kernel: whoever waits for this grid waits for both.  One CTA
     // waiting is enough for that (a grid completes when its last CTA exits); the
-    // others exit at once and leave their SM slots to the kernels chained after
+    // others exit at once and leave their SMs to the kernels chained after
     // this one.
     if (blockIdx.x == 0) grid_dep_wait();
 }
 
 }  // namespace
 
-cudaError_t launch_cache_append(const AppendArgs &a, bool pdl, cudaStream_t stream) {
+cudaError_t launch_cache_append(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const AppendArgs &a, bool pdl,
+                                cudaStream_t stream) {
     const int units = a.n_layers * a.heads * a.nblk;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const int grid = units < 2 * sms ? units : 2 * sms;  // each CTA keeps 64 KB of loads in flight
-    return launch_kernel(cache_append_kernel, dim3(grid), dim3(kThreads), 0, stream, pdl, a);
+    const size_t smem = sizeof(AppendSmem) + 1024;  // + alignment slack
+    if ((e = cudaFuncSetAttribute(cache_append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(smem))) != cudaSuccess)
+        return e;
+    const int grid = units < sms ? units : sms;
+    return launch_kernel(cache_append_kernel, dim3(grid), dim3(kThreads), smem, stream, pdl, tm_k, tm_v, a);
 }
 
 }  // namespace lcsa

@@ -78,15 +78,6 @@ __device__ __forceinline__ int div_by(int n, uint64_t m) {
     return static_cast<int>((static_cast<uint64_t>(static_cast<uint32_t>(n)) * m) >> 32);
 }
 
-// lo += low bf16 of w, hi += high bf16 of w: mixed-precision fp32 adds (the
-// bf16 operand widens exactly, one rounding, as a plain fp32 add would do).
-__device__ __forceinline__ void add_bf16x2(float &lo, float &hi, uint32_t w) {
-    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
-        "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
-        : "+f"(lo), "+f"(hi)
-        : "r"(w));
-}
-
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));

@@ -80,15 +80,19 @@ cudaError_t launch_draft(const DraftArgs &a, bool pdl, cudaStream_t stream);
 
 // Cache append: token layout -> block layout ring slots + k block means.
 struct AppendArgs {
-    const uint16_t *k_tok;
-    const uint16_t *v_tok;
     uint16_t *k_cache;
     uint16_t *v_cache;
     float *kmean;
-    int32_t heads, grid_h, grid_w, nblk, tok_h, tok_w, n_layers;
+    int32_t heads, grid_h, grid_w, nblk, n_layers;
     int32_t slots[kMaxAppendLayers];
+    uint64_t m_nblk, m_heads, m_gw;  // multiply-high multipliers of nblk, heads, grid_w
+    int32_t *status;                 // may be null
+    uint64_t timeout_ns;
 };
 
-cudaError_t launch_cache_append(const AppendArgs &a, bool pdl, cudaStream_t stream);
+// tm_k / tm_v: rank-4 maps over the chunk's k / v in token layout with a
+// (128 dims, 8, 8, 2 frames) box, no swizzle (one box = one block, in block order).
+cudaError_t launch_cache_append(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const AppendArgs &a, bool pdl,
+                                cudaStream_t stream);
 
 }  // namespace lcsa

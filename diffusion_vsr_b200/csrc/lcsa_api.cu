@@ -112,6 +112,24 @@ bool make_token_map(CUtensorMap *m, const void *base, int64_t frames, int tok_h,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Rank-4 map over a chunk's k or v in token layout (dims, x, y, frames) with a
+// whole-block box (128 dims, 8, 8, 2 frames), no swizzle: the box lands in
+// shared memory in block order (intra index (t, y, x) row-major).
+bool make_chunk_map(CUtensorMap *m, const void *base, int64_t frames, int tok_h, int tok_w) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(tok_w),
+                                static_cast<cuuint64_t>(tok_h), static_cast<cuuint64_t>(frames)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHeadDim) * 2,
+                                   static_cast<cuuint64_t>(kHeadDim) * 2 * tok_w,
+                                   static_cast<cuuint64_t>(kHeadDim) * 2 * tok_w * tok_h};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(kHeadDim), 8, 8, 2};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Rank-2 map over a block-layout ring [rows][128] with a (64 dims, 128 rows) box.
 bool make_ring_map(CUtensorMap *m, const void *base, int64_t rows) {
     EncodeTiledFn enc = encode_fn();
@@ -146,7 +164,6 @@ const char *lcsa_status_string(int code) {
 
 int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok, int32_t n_layers, int32_t flags,
                       int32_t *d_status, void *stream) {
-    (void)d_status;  // the append kernel has no device-side failure mode
     int rc = check_cache(cache);
     if (rc != LCSA_OK) return rc;
     if (!k_tok || !v_tok || !aligned16(k_tok) || !aligned16(v_tok)) return LCSA_ERR_INVALID_ARG;
@@ -157,9 +174,19 @@ int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok
     if (pdl && n_layers > cache->capacity - window) return LCSA_ERR_INVALID_ARG;
     if ((rc = check_device()) != LCSA_OK) return rc;
 
+    const int64_t frames = static_cast<int64_t>(cache->heads) * 2 * n_layers;
+    const int64_t units = static_cast<int64_t>(n_layers) * cache->heads * cache->grid_h * cache->grid_w;
+    const int64_t nblk64 = static_cast<int64_t>(cache->grid_h) * cache->grid_w;
+    // unit decomposition by multiply-high division, exact while dividend x divisor <= 2^32
+    if (units * nblk64 > (1ll << 32) || static_cast<int64_t>(n_layers) * cache->heads * cache->heads > (1ll << 32) ||
+        nblk64 * cache->grid_w > (1ll << 32))
+        return LCSA_ERR_INVALID_ARG;
+    CUtensorMap tk, tv;
+    if (!make_chunk_map(&tk, k_tok, frames, 8 * cache->grid_h, 8 * cache->grid_w) ||
+        !make_chunk_map(&tv, v_tok, frames, 8 * cache->grid_h, 8 * cache->grid_w))
+        return LCSA_ERR_CUDA;
+
     lcsa::AppendArgs a{};
-    a.k_tok = static_cast<const uint16_t *>(k_tok);
-    a.v_tok = static_cast<const uint16_t *>(v_tok);
     a.k_cache = static_cast<uint16_t *>(cache->k);
     a.v_cache = static_cast<uint16_t *>(cache->v);
     a.kmean = cache->kmean;
@@ -167,9 +194,12 @@ int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok
     a.grid_h = cache->grid_h;
     a.grid_w = cache->grid_w;
     a.nblk = cache->grid_h * cache->grid_w;
-    a.tok_h = 8 * cache->grid_h;
-    a.tok_w = 8 * cache->grid_w;
     a.n_layers = n_layers;
+    a.m_nblk = lcsa::div_magic_host(static_cast<uint32_t>(a.nblk));
+    a.m_heads = lcsa::div_magic_host(static_cast<uint32_t>(a.heads));
+    a.m_gw = lcsa::div_magic_host(static_cast<uint32_t>(a.grid_w));
+    a.status = d_status;
+    a.timeout_ns = lcsa::kWatchdogNs;
     int oldest = cache->oldest, count = cache->count;
     for (int i = 0; i < n_layers; ++i) {
         a.slots[i] = (oldest + count) % cache->capacity;  // the slot after the newest layer
@@ -179,7 +209,8 @@ int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok
             oldest = (oldest + 1) % cache->capacity;
         }
     }
-    if (lcsa::launch_cache_append(a, pdl, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LCSA_ERR_CUDA;
+    if (lcsa::launch_cache_append(tk, tv, a, pdl, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return LCSA_ERR_CUDA;
     cache->oldest = oldest;
     cache->count = count;
     return LCSA_OK;

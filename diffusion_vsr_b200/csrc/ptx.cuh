@@ -125,6 +125,13 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, uint32_t sr
                  : "memory");
 }
 
+// Plain bulk copy of `bytes` (a multiple of 16) from shared to global memory,
+// tracked by the bulk async-group of the issuing thread.
+__device__ __forceinline__ void bulk_store(void *gdst, uint32_t ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 __device__ __forceinline__ void bulk_wait_group_read0() {
@@ -280,6 +287,15 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bo
         : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
         : "memory");
     return r != 0;
+}
+
+// lo += low bf16 of w, hi += high bf16 of w: mixed-precision fp32 adds (the
+// bf16 operand widens exactly, one rounding, as a plain fp32 add would do).
+__device__ __forceinline__ void add_bf16x2(float &lo, float &hi, uint32_t w) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(w));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -128,8 +128,12 @@ typedef struct lcsa_kv_cache {
  * when `window` layers are resident the oldest is dropped and `oldest`
  * advances (without spare slots its slot is the one reused).
  *   flags: 0 or LCSA_FLAG_PDL (see there).
+ *   d_status: device word (may be NULL); LCSA_ERR_TIMEOUT is OR-ed into it
+ *   when a bounded wait for a copy gave up.
+ * The copies are TMA loads of whole blocks and bulk stores into the ring.
  * Updates cache->oldest/count on the host when the copy is enqueued, so calls
- * on one cache must be serialised by the caller.  1 <= n_layers <= capacity.
+ * on one cache must be serialised by the caller.  1 <= n_layers <= window
+ * (and <= 16).
  */
 int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok,
                       int32_t n_layers, int32_t flags, int32_t *d_status, void *stream);
