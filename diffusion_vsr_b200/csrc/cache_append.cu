@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < n_mine; ++i) {
         const int s = i % kStages;
         ok = mbar_wait(smem_u32(&sm.full[s]), (i / kStages) & 1, abort_word, a.timeout_ns);
+        if (i == 0 && tid == 0 && (a.flags & LCSA_FLAG_FORCE_TIMEOUT)) ok = false;  // test hook
         if (!__syncthreads_and(ok)) {
             ok = false;
             break;

@@ -88,6 +88,7 @@ struct AppendArgs {
     uint64_t m_nblk, m_heads, m_gw;  // multiply-high multipliers of nblk, heads, grid_w
     int32_t *status;                 // may be null
     uint64_t timeout_ns;
+    int32_t flags;
 };
 
 // tm_k / tm_v: rank-4 maps over the chunk's k / v in token layout with a

@@ -200,6 +200,7 @@ int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok
     a.m_gw = lcsa::div_magic_host(static_cast<uint32_t>(a.grid_w));
     a.status = d_status;
     a.timeout_ns = lcsa::kWatchdogNs;
+    a.flags = flags;
     int oldest = cache->oldest, count = cache->count;
     for (int i = 0; i < n_layers; ++i) {
         a.slots[i] = (oldest + count) % cache->capacity;  // the slot after the newest layer

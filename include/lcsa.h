@@ -54,7 +54,9 @@ enum lcsa_status {
 
 /* lcsa_params.flags */
 #define LCSA_FLAG_FORCE_TIMEOUT 1 /* test hook: the first consumer wait of
-                                     lcsa_attention gives up at once */
+                                     lcsa_attention (lcsa_params.flags) or of
+                                     every CTA of lcsa_cache_append (its flags
+                                     argument) gives up at once */
 #define LCSA_FLAG_PDL 2           /* launch as a programmatic dependent of the
                                      kernel that precedes the call in the stream,
                                      so that it starts while that kernel finishes.
@@ -127,7 +129,7 @@ typedef struct lcsa_kv_cache {
  * the slot after the newest layer, together with its fp32 block means of k;
  * when `window` layers are resident the oldest is dropped and `oldest`
  * advances (without spare slots its slot is the one reused).
- *   flags: 0 or LCSA_FLAG_PDL (see there).
+ *   flags: 0, LCSA_FLAG_PDL and/or LCSA_FLAG_FORCE_TIMEOUT (see there).
  *   d_status: device word (may be NULL); LCSA_ERR_TIMEOUT is OR-ed into it
  *   when a bounded wait for a copy gave up.
  * The copies are TMA loads of whole blocks and bulk stores into the ring.

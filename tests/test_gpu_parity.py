@@ -319,6 +319,26 @@ def test_forced_watchdog_expiry_reports_timeout_and_context_survives():
     assert torch.equal(again, ref)
 
 
+def test_cache_append_forced_timeout_reports_status_and_context_survives():
+    """The append's bounded copy waits: a forced expiry is reported, nothing hangs or faults."""
+    L, w, q, k, v, layer = _tiny_setup(topk=8)
+    n = w.q_layers
+    ref = L.KVCache.allocate(n, w.heads, w.grid_h, w.grid_w, device="cuda")
+    L.lcsa_cache_append(ref, k, v)
+    cache = L.KVCache.allocate(n, w.heads, w.grid_h, w.grid_w, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.lcsa_cache_append(cache, k, v, d_status=st, flags=L.LCSA_FLAG_FORCE_TIMEOUT)
+    torch.cuda.synchronize()
+    assert st.item() & L.LCSA_ERR_TIMEOUT
+    # the context is still usable: a normal append gives the reference ring bit for bit
+    cache.reset()
+    st.zero_()
+    L.lcsa_cache_append(cache, k, v, d_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert torch.equal(cache.k, ref.k) and torch.equal(cache.v, ref.v) and torch.equal(cache.kmean, ref.kmean)
+
+
 def test_invalid_arguments_are_rejected():
     L, w, q, k, v, layer = _tiny_setup()
     out = torch.empty_like(q)
