@@ -482,14 +482,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
                 tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
                 tmem_wait_ld();
-                // row maximum: eight independent chains, then a small tree
+                // row maximum: eight independent chains of 3-input maxima, then a small tree
                 float mx8[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(s[e]);
+                for (int e = 0; e < 8; ++e) {
+                    float acc = fmax3(__uint_as_float(s[e]), __uint_as_float(s[8 + e]), __uint_as_float(s[16 + e]));
 #pragma unroll
-                for (int k = 8; k < 128; k += 8) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], __uint_as_float(s[k + e]));
+                    for (int k = 24; k < 120; k += 16)
+                        acc = fmax3(acc, __uint_as_float(s[k + e]), __uint_as_float(s[k + 8 + e]));
+                    mx8[e] = fmaxf(acc, __uint_as_float(s[120 + e]));
                 }
                 const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
@@ -515,22 +516,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_st32(o_addr + cc * 32, o);
                     }
                 }
-                // P = 2^(s*c - m), summed in eight independent chains, packed to bf16
-                // and written over S in four 32-key quarters, each announced as soon
-                // as it is in TMEM so that its PV MMAs can start.
-                float sum8[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
+                // P = 2^(s*c - m) (scale and shift as packed f32x2 FMAs), summed in
+                // eight independent chains (four packed pairs), packed to bf16 and
+                // written over S in four 32-key quarters, each announced as soon as it
+                // is in TMEM so that its PV MMAs can start.
+                const uint64_t c2 = f32x2_pack(c, c), nm2 = f32x2_pack(-m_next, -m_next);
+                uint64_t sum4[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
                         const int col = qq * 32 + 2 * k;
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(s[col]), c, -m_next));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(s[col + 1]), c, -m_next));
-                        sum8[(2 * k) & 7] += p0;
-                        sum8[(2 * k + 1) & 7] += p1;
+                        float x0, x1;
+                        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(s[col]), __uint_as_float(s[col + 1])), c2, nm2),
+                                     x0, x1);
+                        const float p0 = ex2_approx(x0);
+                        const float p1 = ex2_approx(x1);
+                        sum4[k & 3] = f32x2_add(sum4[k & 3], f32x2_pack(p0, p1));
                         pk[k] = pack_bf16x2(p0, p1);
                     }
                     tmem_st16(s_addr + qq * 16, pk);
@@ -539,6 +542,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&sm.bar_pq[qq][w]));
                 }
+                float sum8[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) f32x2_unpack(sum4[e], sum8[2 * e], sum8[2 * e + 1]);
                 const float rs =
                     ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
                 l = l * alpha + rs;
