@@ -584,15 +584,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(tmem + lane_off + col_o(1 - w) + col, o1[cc]);
                 }
                 tmem_wait_ld();
+                if (n_mine > 0 && n_other > 0) {  // (uniform over the CTA) both accumulators hold tiles
+                    const uint64_t fs2 = f32x2_pack(f_self, f_self), fo2 = f32x2_pack(f_oth, f_oth);
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
+                    for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const float a0 = n_mine > 0 ? __uint_as_float(o0[cc][2 * k]) : 0.f;
-                        const float a1 = n_mine > 0 ? __uint_as_float(o0[cc][2 * k + 1]) : 0.f;
-                        const float b0 = n_other > 0 ? __uint_as_float(o1[cc][2 * k]) : 0.f;
-                        const float b1 = n_other > 0 ? __uint_as_float(o1[cc][2 * k + 1]) : 0.f;
-                        pk[cc][k] = pack_bf16x2(a0 * f_self + b0 * f_oth, a1 * f_self + b1 * f_oth);
+                        for (int k = 0; k < 16; ++k) {
+                            const uint64_t b = f32x2_mul(
+                                f32x2_pack(__uint_as_float(o1[cc][2 * k]), __uint_as_float(o1[cc][2 * k + 1])), fo2);
+                            float r0, r1;
+                            f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(o0[cc][2 * k]),
+                                                              __uint_as_float(o0[cc][2 * k + 1])),
+                                                   fs2, b),
+                                         r0, r1);
+                            pk[cc][k] = pack_bf16x2(r0, r1);
+                        }
+                    }
+                } else {
+                    // one accumulator holds the row's tiles (the other one is stale: not read)
+                    const bool mine = n_mine > 0;
+                    const float f = mine ? f_self : f_oth;
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const uint32_t *src = mine ? o0[cc] : o1[cc];
+                            pk[cc][k] = pack_bf16x2(__uint_as_float(src[2 * k]) * f, __uint_as_float(src[2 * k + 1]) * f);
+                        }
                     }
                 }
             }
