@@ -82,13 +82,19 @@ struct __align__(1024) AttnSmem {
     uint64_t bar_pvdone[2];
     uint64_t bar_ofinal;
     uint64_t bar_ofree;
+    uint64_t bar_mlready;  // the early group's (m, l) of the row are in ml_early
+    uint64_t bar_mlfree;   // the late group has read them
     uint64_t bar_drain[2];
     uint64_t bar_info_full[kInfoSlots];
     uint64_t bar_info_empty[kInfoSlots];
     int32_t info_n[kInfoSlots];  // validated kept count of row r in slot r % kInfoSlots
     uint32_t tmem_base;
     int32_t abort_word;
+    float2 ml_early[128];  // (m, l) per query row of the group that finishes a row first
 };
+
+// the layout plus the 1 KB alignment slack fits the 227 KB a CTA may opt into
+static_assert(sizeof(AttnSmem) + 1024 <= 232448, "shared memory layout too large");
 
 __device__ __forceinline__ uint32_t col_s(int w) { return static_cast<uint32_t>(w) * 128u; }
 __device__ __forceinline__ uint32_t col_o(int w) { return 256u + static_cast<uint32_t>(w) * 128u; }
@@ -220,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&sm.bar_qfull[b]), 1);
-            mbar_init(smem_u32(&sm.bar_qempty[b]), 2);  // one arrival per softmax group (its output copy read the buffer)
+            mbar_init(smem_u32(&sm.bar_qempty[b]), 1);  // the late group's output copy read the buffer
             mbar_init(smem_u32(&sm.bar_sfull[b]), 1);
             for (int qq = 0; qq < 4; ++qq) mbar_init(smem_u32(&sm.bar_pq[qq][b]), 4);  // one arrival per warp
             mbar_init(smem_u32(&sm.bar_drain[b]), 1);
@@ -235,7 +241,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&sm.bar_vempty[s]), 1);
         }
         mbar_init(smem_u32(&sm.bar_ofinal), 2);  // one commit per MMA issuer
-        mbar_init(smem_u32(&sm.bar_ofree), 8);
+        mbar_init(smem_u32(&sm.bar_ofree), 4);    // the late group's warps read both accumulators
+        mbar_init(smem_u32(&sm.bar_mlready), 4);  // the early group's warps
+        mbar_init(smem_u32(&sm.bar_mlfree), 4);   // the late group's warps
         for (int i = 0; i < kInfoSlots; ++i) {
             mbar_init(smem_u32(&sm.bar_info_full[i]), 1);
             mbar_init(smem_u32(&sm.bar_info_empty[i]), 10);  // 2 MMA issuers + 8 softmax warps
@@ -440,10 +448,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         for (int unit = blockIdx.x; unit < a.n_units; unit += gridDim.x, ++r) {
             const int is = r % kInfoSlots;
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(smem_u32(&sm.bar_info_full[is]), (r / kInfoSlots) & 1, abort_word, to));
-            // both groups leave together when a wait gave up
-            if (!named_bar_and(1, 256, ok)) {
+            if (ok)
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(smem_u32(&sm.bar_info_full[is]), (r / kInfoSlots) & 1, abort_word, to));
+            // the four warps of the group leave together when a wait gave up
+            // (constant barrier ids: the barrier count stays known)
+            const bool go = !*abort_word;
+            if (!(w == 0 ? named_bar_and(2, 128, ok && go) : named_bar_and(3, 128, ok && go))) {
                 ok = false;
                 break;
             }
@@ -551,40 +562,64 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_used = m_next;
                 if (i == 0 && elected && pending_q >= 0) release_q(pending_q);
             }
+            const int late = (n - 1) & 1;  // the group of the row's last tile runs the epilogue
+            if (w != late) {
+                // ---------------------------------------------- early group
+                // Hand this group's (m, l) of the row to the late group, once that
+                // has read the previous row's, and go on to the next row: its first
+                // tile overlaps the late group's epilogue (its PV waits for the
+                // accumulators to be read, bar_ofree).
+                if (ok && act >= 1)
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(smem_u32(&sm.bar_mlfree), (act - 1) & 1, abort_word, to));
+                if (ok) {
+                    sm.ml_early[row] = make_float2(m_used, l);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&sm.bar_mlready));  // release: ml_early written
+                    if (elected && pending_q >= 0) release_q(pending_q);
+                }
+                ++act;
+                continue;
+            }
+            // -------------------------------------------- late group: epilogue
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_ofinal), act & 1, abort_word, to));
-            // both groups take the same decision on going through the epilogue
-            if (!named_bar_and(1, 256, ok && !*abort_word)) {
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_mlready), act & 1, abort_word, to));
+            // the group's warps take the same decision on going through the epilogue
+            const bool go_epi = !*abort_word;
+            if (!(w == 0 ? named_bar_and(2, 128, ok && go_epi) : named_bar_and(3, 128, ok && go_epi))) {
                 ok = false;
                 break;
             }
-            // ------------------------------------------------------ epilogue
             tc_fence_after();
-            float *mlx = reinterpret_cast<float *>(sm.q[qb]);  // every QK of this row completed
-            mlx[(w * 128 + row) * 2 + 0] = m_used;
-            mlx[(w * 128 + row) * 2 + 1] = l;
-            named_bar_sync(2, 256);
-            const float m_o = mlx[((1 - w) * 128 + row) * 2 + 0];
-            const float l_o = mlx[((1 - w) * 128 + row) * 2 + 1];
+            const float2 mle = sm.ml_early[row];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.bar_mlfree));
+            const float m_o = mle.x, l_o = mle.y;
             const float m = fmaxf(m_used, m_o);
-            const float a_self = n_mine > 0 ? ex2_approx(m_used - m) : 0.f;
+            const float a_self = ex2_approx(m_used - m);  // the late group always holds a tile
             const float a_oth = n_other > 0 ? ex2_approx(m_o - m) : 0.f;
             const float L = l * a_self + l_o * a_oth;
             const float inv_l = L > 0.f ? 1.f / L : 0.f;
             const float f_self = a_self * inv_l, f_oth = a_oth * inv_l;
-            // this group's output dims [64w, 64w+64) of its row, merged and packed to bf16
-            uint32_t pk[2][16];
-            {
-                // both 32-column halves of both accumulators in one TMEM round trip
+            // Both 64-dim halves of the row's output, one at a time: the two
+            // accumulators read, merged, packed to bf16 and staged in the row's Q
+            // buffer (every QK of the row completed), 128-byte swizzled as the TMA
+            // box expects (row = token of the block, 16-byte chunk c of the row at
+            // chunk position c ^ (row & 7)).
+            uint8_t *tile = sm.q[qb];
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[2][16];
                 uint32_t o0[2][32], o1[2][32];
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
-                    const uint32_t col = static_cast<uint32_t>(w * 64 + cc * 32);
-                    // (an accumulator without tiles holds stale data: selected away below)
+                    const uint32_t col = static_cast<uint32_t>(h * 64 + cc * 32);
+                    // (without tiles the early group's accumulator is stale: read, not used)
                     tmem_ld32(tmem + lane_off + col_o(w) + col, o0[cc]);
                     tmem_ld32(tmem + lane_off + col_o(1 - w) + col, o1[cc]);
                 }
                 tmem_wait_ld();
-                if (n_mine > 0 && n_other > 0) {  // (uniform over the CTA) both accumulators hold tiles
+                if (n_other > 0) {  // (uniform over the group) both accumulators hold tiles
                     const uint64_t fs2 = f32x2_pack(f_self, f_self), fo2 = f32x2_pack(f_oth, f_oth);
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
@@ -601,16 +636,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 } else {
-                    // one accumulator holds the row's tiles (the other one is stale: not read)
-                    const bool mine = n_mine > 0;
-                    const float f = mine ? f_self : f_oth;
+                    // the early group had no tile
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const uint32_t *src = mine ? o0[cc] : o1[cc];
-                            pk[cc][k] = pack_bf16x2(__uint_as_float(src[2 * k]) * f, __uint_as_float(src[2 * k + 1]) * f);
-                        }
+                        for (int k = 0; k < 16; ++k)
+                            pk[cc][k] = pack_bf16x2(__uint_as_float(o0[cc][2 * k]) * f_self,
+                                                    __uint_as_float(o0[cc][2 * k + 1]) * f_self);
+                    }
+                }
+                uint8_t *half_buf = tile + h * kHalfBytes;
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+                    for (int qd = 0; qd < 4; ++qd) {
+                        const int chunk = cc * 4 + qd;
+                        *reinterpret_cast<uint4 *>(half_buf + row * 128 + ((chunk ^ (row & 7)) << 4)) =
+                            make_uint4(pk[cc][4 * qd], pk[cc][4 * qd + 1], pk[cc][4 * qd + 2], pk[cc][4 * qd + 3]);
                     }
                 }
             }
@@ -618,31 +660,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ofree));
-            if (w == 0 && a.lse) a.lse[tok] = L > 0.f ? (m + __log2f(L)) * kLn2 : -INFINITY;
-            // every thread has read the (m, l) exchange before the tile overwrites it
-            named_bar_sync(3, 256);
-            // Stage this group's half of the bf16 output tile in the row's Q buffer,
-            // 128-byte swizzled as the TMA box expects (row = token of the block,
-            // 16-byte chunk c of the row at chunk position c ^ (row & 7)), then one
-            // TMA store per group writes it into token layout (reverse partition).
-            uint8_t *half_buf = sm.q[qb] + w * kHalfBytes;
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-#pragma unroll
-                for (int qd = 0; qd < 4; ++qd) {
-                    const int chunk = cc * 4 + qd;
-                    *reinterpret_cast<uint4 *>(half_buf + row * 128 + ((chunk ^ (row & 7)) << 4)) =
-                        make_uint4(pk[cc][4 * qd], pk[cc][4 * qd + 1], pk[cc][4 * qd + 2], pk[cc][4 * qd + 3]);
-                }
-            }
+            if (a.lse) a.lse[tok] = L > 0.f ? (m + __log2f(L)) * kLn2 : -INFINITY;
+            // the staged tile goes out with two TMA stores (one per 64-dim half)
+            // into token layout (the reverse partition)
             fence_proxy_async_smem();
             if (w == 0) named_bar_sync(4, 128);  // (constant ids: the barrier count stays known)
             else named_bar_sync(5, 128);
             if (elected) {
                 if (pending_q >= 0) release_q(pending_q);
-                tma_store_4d(&tm_o, smem_u32(half_buf), 64 * w, rg.qbx * 8, rg.qby * 8, rg.frame0);
+                tma_store_4d(&tm_o, smem_u32(tile), 0, rg.qbx * 8, rg.qby * 8, rg.frame0);
+                tma_store_4d(&tm_o, smem_u32(tile) + kHalfBytes, 64, rg.qbx * 8, rg.qby * 8, rg.frame0);
                 bulk_commit_group();
-                pending_q = qb;  // released once the copy has read it (next row's first tile)
+                pending_q = qb;  // released once the copy has read it (this group's next tile)
             }
             ++act;
         }
