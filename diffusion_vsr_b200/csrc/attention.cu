@@ -31,10 +31,12 @@
 //                  j = w, w+2, ... of a row with its own S and O in TMEM: one
 //                  query row per thread, online softmax in the log2 domain with
 //                  lazy rescaling of O (only when the row maximum grew by more
-//                  than 2^8), P written as bf16 over S.  At the end of a row both
-//                  groups merge (m, l, O); each stages one 64-dim half of the
-//                  bf16 output tile in the row's Q buffer and writes it with one
-//                  TMA store into token layout (the reverse partition).
+//                  than 2^8), P written as bf16 over S.  At the end of a row the
+//                  group holding its last tile merges (m, l, O) of both groups,
+//                  stages the bf16 output tile in the row's Q buffer and writes
+//                  it with two TMA stores into token layout (the reverse
+//                  partition); the other group hands over its (m, l) through
+//                  shared memory and starts the next row at once.
 // TMEM (512 columns): S_w at 128*w, O_w at 256 + 128*w.
 // Launched as a programmatic dependent of the draft mask (LCSA_FLAG_PDL), the
 // set-up overlaps the draft's tail and the producer waits for it before it
