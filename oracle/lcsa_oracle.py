@@ -312,16 +312,20 @@ def lcsa_step(q_tok: np.ndarray, cache: KVCacheModel, grid_h: int, grid_w: int, 
 
 
 def near_tie_rows(scores: np.ndarray, allowed: np.ndarray, mq: np.ndarray, mk: np.ndarray,
-                  topk: int, rel: float = 1e-5) -> np.ndarray:
+                  topk: int, rel: float = 1e-5, scale: str = "dot") -> np.ndarray:
     """Bool [H, Nq]: rows whose top-k boundary is within fp32 noise.
 
     A row is exempt from the bit-exact mask comparison when its k-th and
-    (k+1)-th largest allowed scores differ by at most ``rel`` times the
-    magnitude scale of those two scores.  The scale is the one the rounding
-    error of a dot product is bounded by: sum_d |mq_d * mk_d| / sqrt(D),
-    taking the larger of the two blocks.  Rows with allowed <= topk are never
-    exempt.
+    (k+1)-th largest allowed scores differ by at most ``rel`` times a
+    magnitude scale of those two scores.  ``scale="dot"`` (used for the
+    acceptance test) takes the scale that bounds the rounding error of a dot
+    product, sum_d |mq_d * mk_d| / sqrt(D), the larger of the two blocks (and
+    at least the scores' magnitudes); ``scale="score"`` takes the plain
+    max(|s_k|, |s_k+1|), reported beside it.  Rows with allowed <= topk are
+    never exempt.
     """
+    if scale not in ("dot", "score"):
+        raise ValueError(scale)
     H, Nq, Nk = scores.shape
     d = mq.shape[-1]
     out = np.zeros((H, Nq), dtype=bool)
@@ -333,8 +337,11 @@ def near_tie_rows(scores: np.ndarray, allowed: np.ndarray, mq: np.ndarray, mk: n
             order = np.lexsort((cand, -scores[h, i, cand]))
             a, b = cand[order[topk - 1]], cand[order[topk]]
             sa, sb = scores[h, i, a], scores[h, i, b]
-            mag = max(np.abs(mq[h, i] * mk[h, a]).sum(), np.abs(mq[h, i] * mk[h, b]).sum()) / math.sqrt(d)
-            out[h, i] = abs(sa - sb) <= rel * max(mag, abs(sa), abs(sb))
+            mag = max(abs(sa), abs(sb))
+            if scale == "dot":
+                mag = max(mag, np.abs(mq[h, i] * mk[h, a]).sum() / math.sqrt(d),
+                          np.abs(mq[h, i] * mk[h, b]).sum() / math.sqrt(d))
+            out[h, i] = abs(sa - sb) <= rel * mag
     return out
 
 

@@ -215,6 +215,24 @@ def test_near_tie_exemption():
     assert not O.near_tie_rows(tie, allowed, mq, mk, 3)[0, 0]
 
 
+def test_near_tie_scales_dot_product_bound_versus_plain_scores():
+    # k-th and (k+1)-th scores 0.5 and 0.4999 (gap 1e-4).  Plain score scale:
+    # 1e-5 * 0.5 = 5e-6 < gap, not exempt.  Dot-product scale: the products
+    # mq_d * mk_d are +-100 (they cancel in the score), sum |.| / sqrt(2) = 141.4,
+    # 1e-5 * 141.4 = 1.4e-3 > gap, exempt.
+    mq = np.ones((1, 1, 2))
+    mk = np.array([[[100.0, -100.0], [100.0, -99.0], [100.0, -99.5]]])
+    allowed = np.ones((1, 3), dtype=bool)
+    s = np.array([[[1.0, 0.5, 0.4999]]])
+    assert O.near_tie_rows(s, allowed, mq, mk, 2, scale="dot")[0, 0]
+    assert not O.near_tie_rows(s, allowed, mq, mk, 2, scale="score")[0, 0]
+    # a gap below 1e-5 of the scores themselves is exempt under both
+    s2 = np.array([[[1.0, 0.5, 0.5 - 1e-6]]])
+    assert O.near_tie_rows(s2, allowed, mq, mk, 2, scale="score")[0, 0]
+    with pytest.raises(ValueError):
+        O.near_tie_rows(s, allowed, mq, mk, 2, scale="bogus")
+
+
 def test_valid_topk_accepts_either_side_of_a_tie_only():
     s = np.array([3.0, 1.0, 1.0, 0.0])
     a = np.ones(4, dtype=bool)
