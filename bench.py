@@ -10,12 +10,16 @@ blocks), local range 11, topk 20.
 
 Prints one JSON line.  ``value`` is the effective throughput in TFLOP/s
 counted over kept tiles only (4 * 128^3 flops per tile); ``ms_per_step`` is
-ms per chunk.  ``--impl reference`` times the fp64 CPU oracle on a bounded
-sample of the same workload (rank 0 only).
+ms per chunk.  ``--sweep`` prints one such line per workload instead.
+``--impl reference`` times the fp64 CPU oracle (rank 0 only): each step is
+one whole chunk of a slice of the heads (append, draft and attention of every
+row of those heads), sized so that the run ends within a few minutes.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs an independent
 replica of the layer (LCSA rows are independent, there is no exchange step),
 so the scaling is weak and the barrier/max reduction is the only collective.
+``--gpus N`` without torchrun starts the N processes itself; under torchrun
+WORLD_SIZE must equal N.
 """
 
 from __future__ import annotations
@@ -24,6 +28,7 @@ import argparse
 import hashlib
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -43,9 +48,12 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
+SWEEP = (("768x1280", 0), ("768x1408", 0), ("1536x2688", 0), ("4k", 8), ("4k", 16), ("4k", 32))
+REFERENCE_BUDGET_S = 150.0  # wall-clock budget of a whole reference-arm run (warm-up + timed steps)
+E2E_MIN_STEPS = 50
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -53,14 +61,22 @@ def parse_args():
     ap.add_argument("--impl", default="lcsa", choices=["lcsa", "reference"])
     ap.add_argument("--workload", default="768x1408", choices=sorted(W.WORKLOADS))
     ap.add_argument("--topk", type=int, default=0, help="override the workload's topk")
+    ap.add_argument("--bufs", type=int, default=8,
+                    help="distinct chunk buffers rotated across steps (fewer: a reduced case for ncu captures)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one JSON line per workload (768x1280, 768x1408, 1536x2688, 4K topk 8/16/32)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
+    return ap.parse_args(argv)
+
+
+def workload_of(name: str, topk: int = 0) -> W.Workload:
+    w = W.WORKLOADS[name]
+    return w.with_topk(topk) if topk else w
 
 
 def workload(args) -> W.Workload:
-    w = W.WORKLOADS[args.workload]
-    return w.with_topk(args.topk) if args.topk else w
+    return workload_of(args.workload, args.topk)
 
 
 def peaks():
@@ -162,19 +178,68 @@ def aggregate_tflops(world: int, flops_per_rank_step: float, ms_per_step: float)
     return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
 
 
+def bench_config(w: W.Workload, kept_tiles: int, world: int) -> dict:
+    """The workload a line is measured on; both arms print this same dict."""
+    return {
+        "workload": f"{w.name} streaming chunk, one DiT attention layer",
+        "heads": w.heads, "head_dim": w.head_dim, "query_blocks": w.n_query_blocks, "key_blocks": w.n_key_blocks,
+        "kv_len_layers": w.kv_len, "local_range": w.local_range,
+        "local_mode": "preserved" if w.local_mode == 0 else "truncated", "topk": w.topk,
+        "kept_tiles_per_chunk": kept_tiles, "tflop_per_chunk": round(kept_tiles * W.flops_per_tile() / 1e12, 5),
+        "l2": "inputs larger than L2 (126 MB): distinct chunks' q/k/v rotated across steps, plus the "
+              "resident ring of kv_len + 1 block-layers",
+        "parallelism": f"replicas x{world}" if world > 1 else "single replica",
+    }
+
+
+# ------------------------------------------------------------- launch helpers
+
+def free_port() -> int:
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def launcher_argv(args_argv, gpus: int, port: int):
+    """Command that starts ``gpus`` ranks of this script, one process per GPU."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *args_argv]
+
+
+def check_world(args, env) -> str:
+    """'run' when this process is a rank of a job of --gpus ranks, 'launch' when
+    it should start them itself; raises SystemExit on a mismatch."""
+    if "WORLD_SIZE" not in env:
+        return "launch" if args.gpus > 1 and args.impl == "lcsa" else "run"
+    world = int(env["WORLD_SIZE"])
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}: start one rank per GPU "
+                         f"(torchrun --nproc-per-node {args.gpus}) or pass --gpus {world}")
+    return "run"
+
+
 # ------------------------------------------------------------------ GPU arm
 
-def run_lcsa(args, rank: int, world: int, local_rank: int):
+def unique_kv_bytes(kept_idx: torch.Tensor, kept_cnt: torch.Tensor, n_key_blocks: int) -> int:
+    """Bytes of the distinct K and V tiles the kept lists of one step touch."""
+    H, Nq, topk = kept_idx.shape
+    valid = torch.arange(topk, device=kept_idx.device)[None, None, :] < kept_cnt[:, :, None]
+    flat = torch.where(valid, kept_idx + torch.arange(H, device=kept_idx.device)[:, None, None] * n_key_blocks,
+                       torch.full_like(kept_idx, -1))
+    n = torch.unique(flat[flat >= 0]).numel()
+    return int(n) * 2 * 128 * 128 * 2
+
+
+def measure_lcsa(w: W.Workload, args, world: int, local_rank: int, dev, with_e2e: bool):
     from diffusion_vsr_b200 import lcsa as L
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w = workload(args)
     flop_tile = W.flops_per_tile()
     prefill, steps = W.stream_plan(w)
     # distinct chunk buffers rotated across steps: per-step inputs (q, k, v) plus the
     # 4-layer ring are larger than the 126 MB L2, so no step starts warm
-    n_bufs = max(4, min(8, len(steps)))
+    n_bufs = max(1, args.bufs)
     positions = [w.kv_len + (i % len(steps)) for i in range(n_bufs)]
     host = [W.gen_layers(w, p, w.q_layers) for p in positions]
     chunks = [[t.to(dev) for t in c] for c in host]
@@ -209,6 +274,7 @@ def run_lcsa(args, rank: int, world: int, local_rank: int):
         step(i)
     torch.cuda.synchronize()
     kept_tiles = int(layer.kept_cnt.sum().item())
+    kv_bytes = unique_kv_bytes(layer.kept_idx, layer.kept_cnt, layer.cache.count * w.blocks_per_layer)
     dist = world > 1
     if dist:
         torch.distributed.barrier()
@@ -247,9 +313,14 @@ def run_lcsa(args, rank: int, world: int, local_rank: int):
     q_bytes = H * Nq * 128 * 128 * 2
     draft_bytes = q_bytes + H * w.n_key_blocks * 128 * 4 + H * Nq * (w.topk + 1) * 4
     append_bytes = 2 * 2 * q_bytes + H * nblk * w.q_layers * 128 * 4
+    # the attention's algorithmic DRAM bytes: Q and O once, every distinct kept K/V tile once
+    attn_bytes = 2 * q_bytes + kv_bytes + H * Nq * (w.topk + 1) * 4
     draft_ms = statistics.mean(t_draft)
     append_ms = statistics.mean(t_append)
+    attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9
     traffic = traffic_for("attention.cu", w.name)
+    tensor_frac = attn_tflops / pk["bf16_tflops"]
+    hbm_frac = attn_gbs / pk["hbm_gbs"]
     result = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -264,31 +335,30 @@ def run_lcsa(args, rank: int, world: int, local_rank: int):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16 q/k/v with per-head low-rank block bias; random, no weights)",
-        "config": {
-            "workload": f"{w.name} streaming chunk, one DiT attention layer",
-            "heads": H, "head_dim": 128, "query_blocks": Nq, "key_blocks": w.n_key_blocks,
-            "kv_len_layers": w.kv_len, "local_range": w.local_range, "topk": w.topk,
-            "kept_tiles_per_chunk": kept_tiles, "tflop_per_chunk": round(step_flops / 1e12, 5),
-            "l2": f"inputs larger than L2: {n_bufs} distinct chunk buffers rotated, ring "
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v" + (" with per-head low-rank block bias" if w.lowrank else "")
+                + "; random, no weights)",
+        "config": bench_config(w, kept_tiles, world),
+        "inputs": f"{n_bufs} distinct chunk buffers rotated, ring "
                   f"{(layer.cache.k.numel() + layer.cache.v.numel()) * 2 / 1e6:.0f} MB "
                   f"({layer.cache.desc.capacity} slots, {w.capacity} resident)",
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "launch": "append, draft and attention each as a programmatic dependent of the kernel before "
-                      "it (LCSA_FLAG_PDL; the append writes a spare ring slot and overlaps the previous "
-                      "step's attention); per-kernel times from a separate pass of plain launches",
-        },
+        "launch": "append, draft and attention each as a programmatic dependent of the kernel before it "
+                  "(LCSA_FLAG_PDL; the append writes a spare ring slot and overlaps the previous step's "
+                  "attention); per-kernel times from a separate pass of plain launches",
         "roofline": {
             "kernel": "lcsa_attention (tcgen05 block-sparse attention)",
             "bound": "tensor",
             "achieved": round(attn_tflops, 2),
             "peak": pk["bf16_tflops"],
             "unit": "TFLOP/s",
-            "frac": round(attn_tflops / pk["bf16_tflops"], 4),
+            "frac": round(tensor_frac, 4),
             "peak_source": f"{pk['source']} dense bf16 (burst)",
             "traffic": traffic,
             "algorithmic_flops_per_launch": step_flops,
             "avg_launch_ms": round(attn_ms, 5),
+            "hbm_bound": {"achieved": round(attn_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                          "frac": round(hbm_frac, 4), "algorithmic_bytes_per_launch": attn_bytes,
+                          "bytes": "Q + O + distinct kept K/V tiles + kept lists"},
+            "binding": "tensor" if tensor_frac >= hbm_frac else "hbm",
         },
         "kernels": {
             "attention_ms": round(attn_ms, 5),
@@ -297,15 +367,19 @@ def run_lcsa(args, rank: int, world: int, local_rank: int):
             "cache_append_median_ms": round(statistics.median(t_append), 5),
             "draft_ms": round(draft_ms, 5),
             "draft_gbs": round(draft_bytes / (draft_ms * 1e-3) / 1e9, 1),
+            "draft_bytes": draft_bytes,
             "cache_append_ms": round(append_ms, 5),
             "cache_append_gbs": round(append_bytes / (append_ms * 1e-3) / 1e9, 1),
+            "cache_append_bytes": append_bytes,
             "hbm_peak_gbs": pk["hbm_gbs"],
         },
         "clocks": clocks.summary(),
         "gpu_launches": 3 * args.steps,
     }
-    if not args.no_e2e:
+    if with_e2e:
         result["e2e"] = run_e2e(args, L, layer, host, dev, stream, step_flops, world)
+    del chunks, layer, out
+    torch.cuda.empty_cache()
     return result
 
 
@@ -322,7 +396,7 @@ def run_e2e(args, L, layer, host, dev, stream, step_flops, world):
         q, k, v = pinned[i % n]
         hs.submit(q, k, v, outs_host[i % 2])
 
-    steps = max(5, args.steps // 4)
+    steps = max(E2E_MIN_STEPS, args.steps // 4)
     for i in range(3):
         e2e_step(i)
     hs.drain_into(stream)
@@ -343,53 +417,22 @@ def run_e2e(args, L, layer, host, dev, stream, step_flops, world):
     d2h = outs_host[0].numel() * outs_host[0].element_size()
     return {"value": round(aggregate_tflops(world, step_flops, ms), 3), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "h2d_gbs": round(h2d / (ms * 1e-3) / 1e9, 1),
             "overlap": "H2D of chunk i+1 and D2H of chunk i-1 overlap chunk i's kernels (two copy streams)"}
 
 
+def run_lcsa(args, rank: int, world: int, local_rank: int):
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if args.sweep:
+        out = []
+        for name, topk in SWEEP:
+            out.append(measure_lcsa(workload_of(name, topk), args, world, local_rank, dev, with_e2e=False))
+        return out
+    return [measure_lcsa(workload(args), args, world, local_rank, dev, with_e2e=not args.no_e2e)]
+
+
 # ------------------------------------------------------------ CPU oracle arm
-
-def oracle_prepare(w: W.Workload):
-    """Prefill the oracle's cache model, then time the per-chunk part of one
-    chunk once: append, the full draft (every row), and the oracle's
-    partition of q and gather of the ring."""
-    from oracle import lcsa_oracle as O
-
-    oc = O.KVCacheModel(w.capacity)
-    prefill, steps = W.stream_plan(w)
-    for p in prefill:
-        _, k, v = W.gen_layers(w, p, 1, "kv")
-        oc.append(k.float().numpy(), v.float().numpy())
-    q, k, v = W.gen_layers(w, steps[0], w.q_layers)
-    qf = q.float().numpy()
-    t0 = time.perf_counter()
-    oc.append(k.float().numpy(), v.float().numpy())
-    res = O.lcsa_step(qf, oc, w.grid_h, w.grid_w, w.topk, w.local_range,
-                      "preserved" if w.local_mode == 0 else "truncated", rows=[])
-    qb = O.partition(qf)
-    kb, vb = oc.keys()
-    t_fixed = time.perf_counter() - t0
-    return {"res": res, "qb": qb, "kb": kb, "vb": vb, "t_fixed": t_fixed,
-            "kept_tiles": int(res["kept_cnt"].sum())}
-
-
-def oracle_rows(w: W.Workload, prep, rows_sample: int, seed: int = 0) -> float:
-    """Seconds the oracle takes for the attention of ``rows_sample`` rows of the
-    prepared chunk (every row when rows_sample >= the chunk's rows)."""
-    from oracle import lcsa_oracle as O
-
-    Nq = w.n_query_blocks
-    if rows_sample >= w.heads * Nq:
-        rows = [(h, i) for h in range(w.heads) for i in range(Nq)]
-    else:
-        rng = np.random.default_rng(seed)
-        rows = [(int(rng.integers(w.heads)), int(rng.integers(Nq))) for _ in range(rows_sample)]
-    res, qb, kb, vb = prep["res"], prep["qb"], prep["kb"], prep["vb"]
-    scale = 1 / np.sqrt(128.0)
-    t0 = time.perf_counter()
-    for h, i in rows:
-        O.sparse_attention_row(qb[h, i], kb[h], vb[h], res["kept_idx"][h, i, :res["kept_cnt"][h, i]], scale)
-    return time.perf_counter() - t0, len(rows)
-
 
 def cpu_cores() -> int:
     try:
@@ -402,67 +445,129 @@ def cpu_cores() -> int:
     return len(os.sched_getaffinity(0))
 
 
+class OracleInputs:
+    """Host copies (fp32, exact bf16 values) of a workload's prefill layers and
+    of a few chunk positions, generated once and sliced by head per step."""
+
+    def __init__(self, w: W.Workload, n_positions: int):
+        prefill, steps = W.stream_plan(w)
+        self.prefill = []
+        for p in prefill:
+            _, k, v = W.gen_layers(w, p, 1, "kv")
+            self.prefill.append((k.float().numpy(), v.float().numpy()))
+        self.chunks = []
+        for p in steps[:max(1, n_positions)]:
+            q, k, v = W.gen_layers(w, p, w.q_layers)
+            self.chunks.append(tuple(t.float().numpy() for t in (q, k, v)))
+
+
+def oracle_chunk(w: W.Workload, inputs: OracleInputs, chunk: int, heads: slice):
+    """Seconds the oracle takes for one whole chunk of the heads ``heads``:
+    append of the chunk's k/v into a cache already holding the kv_len prefill
+    layers (the prefill itself is not timed), then the draft and the attention
+    of every row of those heads.  Returns (seconds, kept tiles)."""
+    from oracle import lcsa_oracle as O
+
+    oc = O.KVCacheModel(w.capacity)
+    for k, v in inputs.prefill:
+        oc.append(k[heads], v[heads])
+    q, k, v = (np.ascontiguousarray(t[heads]) for t in inputs.chunks[chunk % len(inputs.chunks)])
+    t0 = time.perf_counter()
+    oc.append(k, v)
+    res = O.lcsa_step(q, oc, w.grid_h, w.grid_w, w.topk, w.local_range,
+                      "preserved" if w.local_mode == 0 else "truncated")
+    dt = time.perf_counter() - t0
+    return dt, int(res["kept_cnt"].sum())
+
+
+def chunk_kept_tiles(w: W.Workload) -> int:
+    """Kept tiles of a steady-state chunk: min(topk, allowed) per row (the
+    oracle's allowed mask), every head."""
+    from oracle import lcsa_oracle as O
+
+    allowed = O.allowed_mask(w.q_layers, w.capacity, w.grid_h, w.grid_w, w.local_range,
+                             "preserved" if w.local_mode == 0 else "truncated")
+    return int(w.heads * np.minimum(allowed.sum(axis=1), w.topk).sum())
+
+
 def cpu_baseline(w: W.Workload, target_s: float = 10.0, max_chunks: int = 4):
-    """The oracle on whole chunks (append, draft and attention of every row),
-    repeated until about ``target_s`` seconds of CPU work."""
-    total_rows = w.heads * w.n_query_blocks
-    spent, est, kept, n = 0.0, 0.0, 0, 0
+    """The oracle on whole chunks (append, draft and attention of every row of
+    every head), repeated until about ``target_s`` seconds of CPU work."""
+    spent, kept, n = 0.0, 0, 0
+    inputs = OracleInputs(w, 2)
     while n < max_chunks and (n == 0 or spent < target_s):
-        prep = oracle_prepare(w)
-        t_rows, _ = oracle_rows(w, prep, total_rows)
-        spent += prep["t_fixed"] + t_rows
-        est += prep["t_fixed"] + t_rows
-        kept += prep["kept_tiles"]
+        dt, kt = oracle_chunk(w, inputs, n, slice(0, w.heads))
+        spent += dt
+        kept += kt
         n += 1
-    value = kept * W.flops_per_tile() / est / 1e12
+    value = kept * W.flops_per_tile() / spent / 1e12
+    total_rows = w.heads * w.n_query_blocks
     return {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-            "ms_per_chunk": round(est / n * 1e3, 1),
+            "ms_per_chunk": round(spent / n * 1e3, 1),
             "sample": f"{n} x one whole chunk: append + draft + attention of all {total_rows} rows, "
                       f"fp64 NumPy oracle",
             "measured_s": round(spent, 2)}
 
 
-def run_reference(args):
-    """The oracle arm: the per-chunk part (append, full draft, partition) is
-    timed once; every step then times the attention of a bounded sample of
-    rows, and a step's time is that part plus the sample scaled to the chunk."""
+def reference_heads_per_step(w: W.Workload, steps: int, warmup: int, t_head_s: float,
+                             budget_s: float = REFERENCE_BUDGET_S) -> int:
+    """Heads per reference step so that (warmup + steps) steps fit ``budget_s``."""
+    per_step = budget_s / max(1, steps + warmup)
+    return int(max(1, min(w.heads, per_step // max(t_head_s, 1e-6))))
+
+
+def run_reference(args, world: int):
+    """The oracle arm.  Each step is the whole chunk for a slice of the heads
+    (every head's cache, draft and attention are independent of the others'):
+    the append, the draft and the attention of every row of those heads, all
+    actually run and timed; the slice width is sized so that the whole run
+    fits a few minutes.  ``value`` = kept-tile flops run / seconds taken."""
     w = workload(args)
-    rows = 16
-    total_rows = w.heads * w.n_query_blocks
-    prep = oracle_prepare(w)
-    ests = []
+    inputs = OracleInputs(w, 2)
+    t_head, _ = oracle_chunk(w, inputs, 0, slice(0, 1))  # probe, not counted
+    nh = reference_heads_per_step(w, args.steps, args.warmup, t_head)
+    times, kept = [], []
     for i in range(args.warmup + args.steps):
-        t_rows, n = oracle_rows(w, prep, rows, seed=i)
+        h0 = (i * nh) % w.heads
+        heads = slice(h0, min(w.heads, h0 + nh))
+        dt, kt = oracle_chunk(w, inputs, i, heads)
         if i >= args.warmup:
-            ests.append(prep["t_fixed"] + t_rows * total_rows / n)
-    est = statistics.mean(ests)
-    kept = prep["kept_tiles"]
-    value = kept * W.flops_per_tile() / est / 1e12
+            times.append(dt)
+            kept.append(kt)
+    total_s = sum(times)
+    value = sum(kept) * W.flops_per_tile() / total_s / 1e12
+    ms_step = total_s / len(times) * 1e3
+    kept_chunk = chunk_kept_tiles(w)
     cores = cpu_cores()
-    sample = (f"per-chunk part (append + draft of all {total_rows} rows) timed once "
-              f"({prep['t_fixed']:.2f} s); per step the attention of {rows} random rows, scaled to the chunk")
+    sample = (f"each step: one whole chunk (append + draft + attention of every row) for {nh} of the "
+              f"{w.heads} heads, fp64 NumPy oracle; ms_per_chunk extrapolates to all heads")
     return {
-        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(est * 1e3, 2),
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 2),
+        "ms_per_chunk": round(ms_step * w.heads / nh, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (same seeded inputs as the CUDA arm)",
-        "config": {"workload": f"{w.name} streaming chunk, one DiT attention layer", "heads": w.heads,
-                   "head_dim": 128, "query_blocks": w.n_query_blocks, "key_blocks": w.n_key_blocks,
-                   "topk": w.topk, "kept_tiles_per_chunk": kept, "parallelism": "host cores"},
+        "config": bench_config(w, kept_chunk, world),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
-def main():
-    args = parse_args()
+def main(argv=None):
+    args = parse_args(argv)
+    mode = check_world(args, os.environ)
+    if mode == "launch":
+        argv_run = list(sys.argv[1:] if argv is None else argv)
+        r = subprocess.run(launcher_argv(argv_run, args.gpus, free_port()))
+        sys.exit(r.returncode)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
+        # the oracle runs once, on rank 0; the other ranks exit without work
         if rank == 0:
-            print(json.dumps(run_reference(args)), flush=True)
+            print(json.dumps(run_reference(args, world)), flush=True)
         return
     if world > 1:
         import datetime
@@ -470,11 +575,12 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        result = run_lcsa(args, rank, world, local_rank)
+        results = run_lcsa(args, rank, world, local_rank)
         if rank == 0:
-            if not args.no_cpu_baseline:
-                result["cpu_baseline"] = cpu_baseline(workload(args))
-            print(json.dumps(result), flush=True)
+            if not args.no_cpu_baseline and not args.sweep:
+                results[0]["cpu_baseline"] = cpu_baseline(workload(args))
+            for r in results:
+                print(json.dumps(r), flush=True)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -704,16 +704,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                             const CUtensorMap &tm_o, const AttnArgs &a, bool pdl, void *out,
+                             const CUtensorMap &tm_o, const AttnArgs &a, bool pdl, void *out, const DeviceInfo &dev,
                              cudaStream_t stream) {
+    static std::atomic<int> smem_set[kMaxDevices];
     const size_t smem = sizeof(AttnSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    const cudaError_t e = ensure_smem_limit(attention_kernel, dev.device, smem, smem_set);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const int grid = a.n_units < sms ? a.n_units : sms;
+    const int grid = a.n_units < dev.sms ? a.n_units : dev.sms;
     return launch_kernel(attention_kernel, dim3(grid), dim3(kThreads), smem, stream, pdl, tm_q, tm_k, tm_v, tm_o, a,
                          static_cast<uint16_t *>(out));
 }

@@ -109,7 +109,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
         }
         const Unit un = unit_of(a, static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x));
-        const size_t blk = (static_cast<size_t>(a.slots[un.li]) * a.heads + un.h) * a.nblk + un.b;
+        int slot = a.first_slot + un.li;  // < 2 * capacity
+        if (slot >= a.capacity) slot -= a.capacity;
+        const size_t blk = (static_cast<size_t>(slot) * a.heads + un.h) * a.nblk + un.b;
         // k mean: this thread sums its 64 tokens of two dimensions
         const uint32_t *kw = reinterpret_cast<const uint32_t *>(sm.k[s]) + half * 64 * (kHeadDim / 2) + pr;
         float lo = 0.f, hi = 0.f;
@@ -157,17 +159,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_cache_append(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const AppendArgs &a, bool pdl,
-                                cudaStream_t stream) {
+                                const DeviceInfo &dev, cudaStream_t stream) {
+    static std::atomic<int> smem_set[kMaxDevices];
     const int units = a.n_layers * a.heads * a.nblk;
-    int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const size_t smem = sizeof(AppendSmem) + 1024;  // + alignment slack
-    if ((e = cudaFuncSetAttribute(cache_append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(smem))) != cudaSuccess)
-        return e;
-    const int grid = units < sms ? units : sms;
+    const cudaError_t e = ensure_smem_limit(cache_append_kernel, dev.device, smem, smem_set);
+    if (e != cudaSuccess) return e;
+    const int grid = units < dev.sms ? units : dev.sms;
     return launch_kernel(cache_append_kernel, dim3(grid), dim3(kThreads), smem, stream, pdl, tm_k, tm_v, a);
 }
 

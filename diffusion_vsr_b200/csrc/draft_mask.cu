@@ -233,10 +233,10 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
             }
         }
     };
-    // Candidates of the layers resident before the chunk (logical layers below
-    // count - q_layers, written by earlier appends) are scored at once; those of
-    // the chunk's own layers only after the wait below.
-    const int c_split = min(ncand, max(a.count - a.q_layers, 0) * wsz);
+    // Candidates of the layers resident before the chunk's append (logical
+    // layers below count - fresh_layers, written by earlier, completed appends)
+    // are scored at once; those of the newest layers only after the wait below.
+    const int c_split = min(ncand, max(a.count - a.fresh_layers, 0) * wsz);
     score_range(0, c_split);
     // Launched as a programmatic dependent of the cache append of the chunk:
     // the key means of its layers are read only from here on (returns at once
@@ -337,12 +337,12 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
 
 }  // namespace
 
-cudaError_t launch_draft(const DraftArgs &a, bool pdl, cudaStream_t stream) {
+cudaError_t launch_draft(const DraftArgs &a, bool pdl, const DeviceInfo &dev, cudaStream_t stream) {
+    static std::atomic<int> smem_set[kMaxDevices];
     const int rows = a.heads * a.q_layers * a.nblk;
     const size_t smem = 4 * static_cast<size_t>(a.cand_cap);
     if (smem > 48 * 1024 - sizeof(DraftSmem)) {
-        cudaError_t e = cudaFuncSetAttribute(draft_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
+        const cudaError_t e = ensure_smem_limit(draft_kernel, dev.device, smem, smem_set);
         if (e != cudaSuccess) return e;
     }
     return launch_kernel(draft_kernel, dim3(rows), dim3(kThreads), smem, stream, pdl, a);

@@ -1,12 +1,45 @@
 // Kernel argument blocks and launchers shared by the C-ABI layer and the kernels.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <utility>
 
 namespace lcsa {
+
+constexpr int kMaxDevices = 64;
+
+// Facts about the current device, queried once per device and process: the
+// LCSA status of its compute capability (only 10.0 is supported) and its SM
+// count.  Returns null when the device cannot be queried.
+struct DeviceInfo {
+    int device;
+    int status;  // LCSA_OK or LCSA_ERR_UNSUPPORTED_DEVICE
+    int sms;
+};
+const DeviceInfo *current_device_info();
+
+// Raises the dynamic shared memory limit of `kernel` on `dev` to `bytes`,
+// calling the runtime only when the limit set so far on that device is lower.
+// `done` holds the limit set so far per device (one array per kernel).
+template <typename Kernel>
+cudaError_t ensure_smem_limit(Kernel kernel, int dev, size_t bytes, std::atomic<int> (&done)[kMaxDevices]) {
+    if (dev < 0 || dev >= kMaxDevices) {
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    }
+    if (done[dev].load(std::memory_order_acquire) >= static_cast<int>(bytes)) return cudaSuccess;
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (e == cudaSuccess) {
+        int cur = done[dev].load(std::memory_order_relaxed);
+        while (cur < static_cast<int>(bytes) &&
+               !done[dev].compare_exchange_weak(cur, static_cast<int>(bytes), std::memory_order_release)) {
+        }
+    }
+    return e;
+}
 
 // Launch of `kernel` on `stream`, optionally as a programmatic dependent of the
 // stream's preceding kernel (it may start before that kernel completes and
@@ -29,7 +62,6 @@ cudaError_t launch_kernel(void (*kernel)(Params...), dim3 grid, dim3 block, size
 
 constexpr int kBlockTokens = 128;
 constexpr int kHeadDim = 128;
-constexpr int kMaxAppendLayers = 16;
 constexpr int kMaxCandidates = 4096;
 constexpr uint64_t kWatchdogNs = 4000000000ull;  // 4 s per bounded wait
 
@@ -57,7 +89,8 @@ struct AttnArgs {
 inline uint64_t div_magic_host(uint32_t d) { return ((1ull << 32) + d - 1) / d; }
 
 cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                             const CUtensorMap &tm_o, const AttnArgs &a, bool pdl, void *out, cudaStream_t stream);
+                             const CUtensorMap &tm_o, const AttnArgs &a, bool pdl, void *out, const DeviceInfo &dev,
+                             cudaStream_t stream);
 
 // Draft mask: q block means, scores over allowed candidates, top-k.
 struct DraftArgs {
@@ -65,6 +98,7 @@ struct DraftArgs {
     const float *kmean;    // [cap][H][nblk][128]
     int32_t heads, grid_h, grid_w, nblk, q_layers, tq, tok_h, tok_w;
     int32_t capacity, oldest, count;
+    int32_t fresh_layers;  // newest layers the preceding kernel may still be writing (PDL)
     int32_t local_range, local_mode, topk;
     int32_t cand_cap;      // most allowed candidates of a row, rounded up to 32
     uint64_t m_nq, m_nblk, m_gw;  // multiply-high multipliers of q_layers*nblk, nblk, grid_w
@@ -76,7 +110,7 @@ struct DraftArgs {
     int32_t *status;
 };
 
-cudaError_t launch_draft(const DraftArgs &a, bool pdl, cudaStream_t stream);
+cudaError_t launch_draft(const DraftArgs &a, bool pdl, const DeviceInfo &dev, cudaStream_t stream);
 
 // Cache append: token layout -> block layout ring slots + k block means.
 struct AppendArgs {
@@ -84,7 +118,7 @@ struct AppendArgs {
     uint16_t *v_cache;
     float *kmean;
     int32_t heads, grid_h, grid_w, nblk, n_layers;
-    int32_t slots[kMaxAppendLayers];
+    int32_t first_slot, capacity;    // layer i of the chunk goes to slot (first_slot + i) % capacity
     uint64_t m_nblk, m_heads, m_gw;  // multiply-high multipliers of nblk, heads, grid_w
     int32_t *status;                 // may be null
     uint64_t timeout_ns;
@@ -94,6 +128,6 @@ struct AppendArgs {
 // tm_k / tm_v: rank-4 maps over the chunk's k / v in token layout with a
 // (128 dims, 8, 8, 2 frames) box, no swizzle (one box = one block, in block order).
 cudaError_t launch_cache_append(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const AppendArgs &a, bool pdl,
-                                cudaStream_t stream);
+                                const DeviceInfo &dev, cudaStream_t stream);
 
 }  // namespace lcsa

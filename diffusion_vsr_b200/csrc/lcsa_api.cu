@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include <cuda.h>
@@ -35,16 +36,43 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Only compute capability 10.0 (B200, sm_100a code) is supported.
-int check_device() {
+}  // namespace
+
+namespace lcsa {
+
+// Facts about the current device, queried once per device (compute capability
+// 10.0 = B200, sm_100a code, and the SM count).
+const DeviceInfo *current_device_info() {
+    static DeviceInfo infos[kMaxDevices];
+    static std::atomic<bool> ready[kMaxDevices];
+    static std::mutex mu;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return LCSA_ERR_CUDA;
-    int major = 0, minor = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-        return LCSA_ERR_CUDA;
-    if (major != 10 || minor != 0) return LCSA_ERR_UNSUPPORTED_DEVICE;
-    return LCSA_OK;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (ready[dev].load(std::memory_order_acquire)) return &infos[dev];
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ready[dev].load(std::memory_order_relaxed)) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return nullptr;  // not cached: the next call queries again
+        infos[dev].device = dev;
+        infos[dev].status = (major == 10 && minor == 0) ? LCSA_OK : LCSA_ERR_UNSUPPORTED_DEVICE;
+        infos[dev].sms = sms;
+        ready[dev].store(true, std::memory_order_release);
+    }
+    return &infos[dev];
+}
+
+}  // namespace lcsa
+
+namespace {
+
+// The current device's facts, or an LCSA status when it cannot be used.
+int device_of(const lcsa::DeviceInfo **info) {
+    *info = lcsa::current_device_info();
+    if (!*info) return LCSA_ERR_CUDA;
+    return (*info)->status;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -58,6 +86,7 @@ int check_cache(const lcsa_kv_cache *c) {
     if (c->window < 0 || c->window > c->capacity) return LCSA_ERR_INVALID_ARG;
     if (c->count < 0 || c->count > window_of(c) || c->oldest < 0 || c->oldest >= c->capacity)
         return LCSA_ERR_INVALID_ARG;
+    if (c->appended < 0 || c->appended > c->capacity) return LCSA_ERR_INVALID_ARG;
     // every token row index of the ring must fit a signed 32-bit TMA coordinate
     const int64_t rows = static_cast<int64_t>(c->capacity) * c->heads * c->grid_h * c->grid_w * kBlockTokens;
     if (rows >= (int64_t(1) << 31)) return LCSA_ERR_INVALID_ARG;
@@ -94,10 +123,46 @@ int64_t max_candidates(const lcsa_params *p, const lcsa_kv_cache *c) {
     return static_cast<int64_t>(c->count) * span(p->grid_h) * span(p->grid_w);
 }
 
+// Small per-thread cache of encoded tensor maps: a streaming caller passes the
+// same buffers call after call, so their maps are encoded once.  Key: the kind
+// of map, the base address and the extents.
+enum MapKind { kTokenMap = 1, kChunkMap = 2, kRingMap = 3 };
+struct MapKey {
+    int kind;
+    const void *base;
+    int64_t a, b, c;
+    bool operator==(const MapKey &o) const {
+        return kind == o.kind && base == o.base && a == o.a && b == o.b && c == o.c;
+    }
+};
+constexpr int kMapCacheSize = 16;
+struct MapCache {
+    MapKey key[kMapCacheSize] = {};
+    CUtensorMap map[kMapCacheSize];
+    int next = 0;
+};
+
+template <typename Encode>
+bool cached_map(CUtensorMap *m, const MapKey &k, Encode encode) {
+    thread_local MapCache cache;
+    for (int i = 0; i < kMapCacheSize; ++i) {
+        if (cache.key[i].kind != 0 && cache.key[i] == k) {
+            *m = cache.map[i];
+            return true;
+        }
+    }
+    if (!encode(m)) return false;
+    const int slot = cache.next;
+    cache.next = (cache.next + 1) % kMapCacheSize;
+    cache.key[slot] = k;
+    cache.map[slot] = *m;
+    return true;
+}
+
 // Rank-4 map over a token-layout bf16 tensor [H*T][8gh][8gw][128] with a
 // (64 dims, 8, 8, 2 frames) box and 128-byte swizzle: one box pair is one
 // (2,8,8) window block, so the partition is done by the copy engine.
-bool make_token_map(CUtensorMap *m, const void *base, int64_t frames, int tok_h, int tok_w) {
+bool encode_token_map(CUtensorMap *m, const void *base, int64_t frames, int tok_h, int tok_w) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(tok_w),
@@ -115,7 +180,7 @@ bool make_token_map(CUtensorMap *m, const void *base, int64_t frames, int tok_h,
 // Rank-4 map over a chunk's k or v in token layout (dims, x, y, frames) with a
 // whole-block box (128 dims, 8, 8, 2 frames), no swizzle: the box lands in
 // shared memory in block order (intra index (t, y, x) row-major).
-bool make_chunk_map(CUtensorMap *m, const void *base, int64_t frames, int tok_h, int tok_w) {
+bool encode_chunk_map(CUtensorMap *m, const void *base, int64_t frames, int tok_h, int tok_w) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(tok_w),
@@ -131,7 +196,7 @@ bool make_chunk_map(CUtensorMap *m, const void *base, int64_t frames, int tok_h,
 }
 
 // Rank-2 map over a block-layout ring [rows][128] with a (64 dims, 128 rows) box.
-bool make_ring_map(CUtensorMap *m, const void *base, int64_t rows) {
+bool encode_ring_map(CUtensorMap *m, const void *base, int64_t rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows)};
@@ -143,11 +208,24 @@ bool make_ring_map(CUtensorMap *m, const void *base, int64_t rows) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_token_map(CUtensorMap *m, const void *base, int64_t frames, int tok_h, int tok_w) {
+    return cached_map(m, MapKey{kTokenMap, base, frames, tok_h, tok_w},
+                      [&](CUtensorMap *o) { return encode_token_map(o, base, frames, tok_h, tok_w); });
+}
+bool make_chunk_map(CUtensorMap *m, const void *base, int64_t frames, int tok_h, int tok_w) {
+    return cached_map(m, MapKey{kChunkMap, base, frames, tok_h, tok_w},
+                      [&](CUtensorMap *o) { return encode_chunk_map(o, base, frames, tok_h, tok_w); });
+}
+bool make_ring_map(CUtensorMap *m, const void *base, int64_t rows) {
+    return cached_map(m, MapKey{kRingMap, base, rows, 0, 0},
+                      [&](CUtensorMap *o) { return encode_ring_map(o, base, rows); });
+}
+
 }  // namespace
 
 extern "C" {
 
-int lcsa_version(void) { return 100; }
+int lcsa_version(void) { return 101; }
 
 const char *lcsa_status_string(int code) {
     switch (code) {
@@ -168,11 +246,12 @@ int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok
     if (rc != LCSA_OK) return rc;
     if (!k_tok || !v_tok || !aligned16(k_tok) || !aligned16(v_tok)) return LCSA_ERR_INVALID_ARG;
     const int window = window_of(cache);
-    if (n_layers < 1 || n_layers > window || n_layers > lcsa::kMaxAppendLayers) return LCSA_ERR_INVALID_ARG;
+    if (n_layers < 1 || n_layers > window) return LCSA_ERR_INVALID_ARG;
     const bool pdl = (flags & LCSA_FLAG_PDL) != 0;
     // overlapping the previous step is safe only while the new layers go to spare slots
     if (pdl && n_layers > cache->capacity - window) return LCSA_ERR_INVALID_ARG;
-    if ((rc = check_device()) != LCSA_OK) return rc;
+    const lcsa::DeviceInfo *dev = nullptr;
+    if ((rc = device_of(&dev)) != LCSA_OK) return rc;
 
     const int64_t frames = static_cast<int64_t>(cache->heads) * 2 * n_layers;
     const int64_t units = static_cast<int64_t>(n_layers) * cache->heads * cache->grid_h * cache->grid_w;
@@ -201,19 +280,17 @@ int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok
     a.status = d_status;
     a.timeout_ns = lcsa::kWatchdogNs;
     a.flags = flags;
-    int oldest = cache->oldest, count = cache->count;
-    for (int i = 0; i < n_layers; ++i) {
-        a.slots[i] = (oldest + count) % cache->capacity;  // the slot after the newest layer
-        if (count < window) {
-            ++count;
-        } else {  // window full: the oldest layer is dropped
-            oldest = (oldest + 1) % cache->capacity;
-        }
-    }
-    if (lcsa::launch_cache_append(tk, tv, a, pdl, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    // each new layer goes to the slot after the newest one (layer i of the chunk
+    // to first_slot + i); once `window` layers are resident the oldest is dropped
+    a.first_slot = (cache->oldest + cache->count) % cache->capacity;
+    a.capacity = cache->capacity;
+    const int count = std::min(window, cache->count + n_layers);
+    const int oldest = (cache->oldest + (cache->count + n_layers - count)) % cache->capacity;
+    if (lcsa::launch_cache_append(tk, tv, a, pdl, *dev, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LCSA_ERR_CUDA;
     cache->oldest = oldest;
     cache->count = count;
+    cache->appended = n_layers;
     return LCSA_OK;
 }
 
@@ -225,7 +302,8 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
     if (!q_tok || !aligned16(q_tok) || !kept_idx || !kept_cnt) return LCSA_ERR_INVALID_ARG;
     const int64_t cand = max_candidates(p, cache);
     if (cand > lcsa::kMaxCandidates) return LCSA_ERR_INVALID_ARG;
-    if ((rc = check_device()) != LCSA_OK) return rc;
+    const lcsa::DeviceInfo *dev = nullptr;
+    if ((rc = device_of(&dev)) != LCSA_OK) return rc;
 
     lcsa::DraftArgs a{};
     a.q = static_cast<const uint16_t *>(q_tok);
@@ -241,6 +319,9 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
     a.capacity = cache->capacity;
     a.oldest = cache->oldest;
     a.count = cache->count;
+    // chained after an append (LCSA_FLAG_PDL), the layers it wrote are read only
+    // after waiting for it: the query layers, and every layer of that append
+    a.fresh_layers = std::max(p->q_layers, cache->appended);
     a.local_range = p->local_range;
     a.local_mode = p->local_mode;
     a.topk = p->topk;
@@ -260,7 +341,7 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
     a.scores = scores_opt;
     a.qmean = qmean_opt;
     a.status = d_status;
-    if (lcsa::launch_draft(a, (p->flags & LCSA_FLAG_PDL) != 0, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (lcsa::launch_draft(a, (p->flags & LCSA_FLAG_PDL) != 0, *dev, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LCSA_ERR_CUDA;
     return LCSA_OK;
 }
@@ -273,7 +354,8 @@ int lcsa_attention(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache 
     if (!q_tok || !out_tok || !aligned16(q_tok) || !aligned16(out_tok) || !kept_idx || !kept_cnt)
         return LCSA_ERR_INVALID_ARG;
     if (q_tok == out_tok) return LCSA_ERR_INVALID_ARG;
-    if ((rc = check_device()) != LCSA_OK) return rc;
+    const lcsa::DeviceInfo *dev = nullptr;
+    if ((rc = device_of(&dev)) != LCSA_OK) return rc;
 
     const int nblk = p->grid_h * p->grid_w;
     const int64_t frames = static_cast<int64_t>(p->heads) * 2 * p->q_layers;
@@ -311,7 +393,7 @@ int lcsa_attention(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache 
     a.m_nq = lcsa::div_magic_host(static_cast<uint32_t>(nq));
     a.m_nblk = lcsa::div_magic_host(static_cast<uint32_t>(nblk));
     a.m_gw = lcsa::div_magic_host(static_cast<uint32_t>(p->grid_w));
-    if (lcsa::launch_attention(tq, tk, tv, to, a, (p->flags & LCSA_FLAG_PDL) != 0, out_tok,
+    if (lcsa::launch_attention(tq, tk, tv, to, a, (p->flags & LCSA_FLAG_PDL) != 0, out_tok, *dev,
                                static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LCSA_ERR_CUDA;
     return LCSA_OK;

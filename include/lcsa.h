@@ -64,14 +64,16 @@ enum lcsa_status {
                                      kernel (griddepcontrol.wait) before reading
                                      the ring, the kept lists or the key means of
                                      the newest q_layers layers, but read q_tok
-                                     (and the draft the key means of the older
-                                     layers) before the wait: set the flag only
-                                     when the preceding kernel writes none of these
-                                     (nor, for lcsa_attention, out_tok or lse_opt),
-                                     e.g. when it is the cache append of the same
-                                     chunk (before the draft: it writes only the
-                                     chunk's own, newest layers) or the draft
-                                     (before the attention).  lcsa_cache_append (flags
+                                     (and the draft the key means of the layers
+                                     older than the newest max(q_layers,
+                                     cache->appended)) before the wait: set the
+                                     flag only when the preceding kernel writes
+                                     none of these (nor, for lcsa_attention,
+                                     out_tok or lse_opt), e.g. when it is the
+                                     cache append of the same chunk (before the
+                                     draft: it writes only the cache->appended
+                                     newest layers) or the draft (before the
+                                     attention).  lcsa_cache_append (flags
                                      argument) writes the ring before the wait and
                                      waits only at its end: set it only when the
                                      preceding kernel writes neither k_tok nor v_tok
@@ -119,6 +121,9 @@ typedef struct lcsa_kv_cache {
     int32_t grid_h;
     int32_t grid_w;
     int32_t window;   /* 0 < window <= capacity, or 0 for capacity */
+    int32_t appended; /* layers written by the last lcsa_cache_append (set by
+                         it; start from 0): a draft chained after that append
+                         (LCSA_FLAG_PDL) reads them only after waiting for it */
 } lcsa_kv_cache;
 
 /*
@@ -133,9 +138,9 @@ typedef struct lcsa_kv_cache {
  *   d_status: device word (may be NULL); LCSA_ERR_TIMEOUT is OR-ed into it
  *   when a bounded wait for a copy gave up.
  * The copies are TMA loads of whole blocks and bulk stores into the ring.
- * Updates cache->oldest/count on the host when the copy is enqueued, so calls
- * on one cache must be serialised by the caller.  1 <= n_layers <= window
- * (and <= 16).
+ * Updates cache->oldest/count/appended on the host when the copy is enqueued,
+ * so calls on one cache must be serialised by the caller.
+ * 1 <= n_layers <= window.
  */
 int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok,
                       int32_t n_layers, int32_t flags, int32_t *d_status, void *stream);

@@ -20,6 +20,11 @@ MODES = {0: "preserved", 1: "truncated"}
 ATOL_OUT = 2e-2      # max-abs error of bf16 outputs against the fp64 oracle
 RTOL_L2_OUT = 5e-3   # relative L2 error of bf16 outputs against the fp64 oracle
 NEAR_TIE_REL = 1e-5
+# Largest share of near-tie rows a workload may exempt from the bit-exact mask
+# comparison.  Observed with the seeded inputs (oracle only, every row of every
+# step the GPU tests run): at most 31 of 3,024 rows (1.0 %, 1536x2688, second
+# chunk); 28 of 6,120 at 4K topk 16; 2 of 792 at 768x1408.
+MAX_EXEMPT_FRAC = 0.015
 
 
 def f32(t: torch.Tensor) -> np.ndarray:
@@ -57,14 +62,18 @@ class StepResult:
     lse_oracle_mask: np.ndarray   # [H, Nq, 128]
     rows: List[Tuple[int, int]]
     exempt: np.ndarray
+    exempt_score_scale: int       # rows exempt under the plain max(|s_k|, |s_k+1|) scale (reported)
     status: int
     ring_ok: Optional[bool] = None
     kmean_err: Optional[float] = None
 
 
 def run_stream(w: W.Workload, n_steps: Optional[int] = None, n_rows: Optional[int] = None,
-               check_ring: bool = False, seed_rows: int = 0) -> List[StepResult]:
-    """Run prefill + steps of ``w`` on the GPU and the oracle side by side."""
+               check_ring: bool = False, seed_rows: int = 0, on_step=None) -> List[StepResult]:
+    """Run prefill + steps of ``w`` on the GPU and the oracle side by side.
+
+    n_rows None compares the attention of every row.  With ``on_step`` each
+    step's result is handed to it and not kept (large workloads)."""
     from diffusion_vsr_b200 import lcsa as L
 
     dev = torch.device("cuda")
@@ -79,8 +88,13 @@ def run_stream(w: W.Workload, n_steps: Optional[int] = None, n_rows: Optional[in
     results = []
     for p in steps[: (n_steps or len(steps))]:
         q, k, v = W.gen_layers(w, p, w.q_layers)
-        results.append(step_both(w, layer.cache, ocache, layer.params, q, k, v, n_rows, check_ring,
-                                 seed_rows + p, p, layer.status))
+        res = step_both(w, layer.cache, ocache, layer.params, q, k, v, n_rows, check_ring,
+                        seed_rows + p, p, layer.status)
+        if on_step is not None:
+            on_step(res)
+            del res
+        else:
+            results.append(res)
     return results
 
 
@@ -143,6 +157,8 @@ def step_both(w: W.Workload, cache, ocache: O.KVCacheModel, params, q, k, v, n_r
     L.lcsa_attention(params, qd, cache, kept_o, cnt_o, out_o, lse_o, d_status=status)
     torch.cuda.synchronize()
     exempt = O.near_tie_rows(ref["scores"], ref["allowed"], ref["mq"], ref["mk"], w.topk, NEAR_TIE_REL)
+    exempt_score = O.near_tie_rows(ref["scores"], ref["allowed"], ref["mq"], ref["mk"], w.topk, NEAR_TIE_REL,
+                                   scale="score")
     return StepResult(
         position=position, oracle=ref,
         gpu_kept=kept.cpu().numpy(), gpu_cnt=cnt.cpu().numpy(),
@@ -150,7 +166,8 @@ def step_both(w: W.Workload, cache, ocache: O.KVCacheModel, params, q, k, v, n_r
         out_pipeline=O.partition(f32(out_p)), out_oracle_mask=O.partition(f32(out_o)),
         lse_oracle_mask=O.partition(lse_o.cpu().numpy()[..., None])[..., 0],
         rows=rows if rows is not None else all_rows,
-        exempt=exempt, status=int(status.item()), ring_ok=ring_ok, kmean_err=kmean_err)
+        exempt=exempt, exempt_score_scale=int(exempt_score.sum()), status=int(status.item()), ring_ok=ring_ok,
+        kmean_err=kmean_err)
 
 
 def ring_matches(cache, ocache: O.KVCacheModel) -> Tuple[bool, float]:
@@ -182,8 +199,8 @@ def check_mask(res: StepResult, w: W.Workload) -> Tuple[int, int, int]:
                 n_exempt += 1
                 sr = ref["scores"][h, i]
                 cand = np.nonzero(ref["allowed"][i])[0]
-                # same scale as the exemption rule: |mq| |mk| / sqrt(D) bounds sum |mq_d mk_d| / sqrt(D)
-                mag = np.linalg.norm(ref["mq"][h, i]) * np.linalg.norm(ref["mk"][h, cand], axis=1).max()
+                # the exemption rule's scale, sum_d |mq_d mk_d| / sqrt(D), largest over the row's candidates
+                mag = np.abs(ref["mq"][h, i][None, :] * ref["mk"][h, cand]).sum(axis=1).max()
                 tol = NEAR_TIE_REL * mag / math.sqrt(ref["mq"].shape[-1])
                 if not O.valid_topk(g, sr, ref["allowed"][i], w.topk, tol):
                     bad += 1

@@ -24,7 +24,7 @@ def _lib():
     return lcsa
 
 
-def _check_step(res, w, require_rows_exact=True):
+def _check_step(res, w):
     ref = res.oracle
     assert res.status == 0, _lib().status_string(res.status)
     # q block means and fp32 draft scores against fp64
@@ -38,9 +38,11 @@ def _check_step(res, w, require_rows_exact=True):
     assert np.all(err <= 1e-5 * mag[:, allowed] + 1e-9)
     # kept sets
     exact, exempt, bad = Hn.check_mask(res, w)
+    print(f"[parity] {w.name} position {res.position}: {exact + exempt} rows, {exact} compared bit-exactly, "
+          f"{exempt} near-tie exempt (dot-product scale; {res.exempt_score_scale} under the plain score scale), "
+          f"{len(res.rows)} attention rows against fp64")
     assert bad == 0, f"{bad} rows differ ({exact} exact, {exempt} near-tie)"
-    if require_rows_exact:
-        assert exact > 0.9 * (exact + exempt)
+    assert exempt <= Hn.MAX_EXEMPT_FRAC * (exact + exempt), (exempt, exact)
     # attention with the oracle's mask
     hs, iis = zip(*res.rows)
     g = res.out_oracle_mask[list(hs), list(iis)]
@@ -84,26 +86,49 @@ def test_768x1280_full_parity():
 
 
 def test_768x1408_streaming_eight_chunks():
+    # every row of all 8 chunks; from the second chunk on the oldest layer is dropped
     w = W.WORKLOADS["768x1408"]
-    results = Hn.run_stream(w, n_rows=24, check_ring=True)
-    assert len(results) == 8
-    for res in results:
+    seen = []
+
+    def check(res):
         assert res.ring_ok and res.kmean_err <= 1e-6
+        assert len(res.rows) == w.heads * w.n_query_blocks
         _check_step(res, w)
+        seen.append(res.position)
+
+    Hn.run_stream(w, check_ring=True, on_step=check)
+    assert len(seen) == 8
 
 
-def test_1536x2688_sampled():
+def test_1536x2688_all_rows_with_eviction():
+    # two chunks, every row; the second chunk's append drops the oldest layer
     w = W.WORKLOADS["1536x2688"]
-    for res in Hn.run_stream(w, n_steps=2, n_rows=16, check_ring=True):
+    seen = []
+
+    def check(res):
         assert res.ring_ok
+        assert len(res.rows) == w.heads * w.n_query_blocks
         _check_step(res, w)
+        seen.append(res.position)
+
+    Hn.run_stream(w, n_steps=2, check_ring=True, on_step=check)
+    assert len(seen) == 2
 
 
 @pytest.mark.parametrize("topk", W.FOURK_TOPK_SWEEP)
-def test_4k_sampled(topk):
+def test_4k_all_rows(topk):
+    # every row; at topk 16 a second, evicting chunk as well
     w = W.WORKLOADS["4k"].with_topk(topk)
-    for res in Hn.run_stream(w, n_steps=1, n_rows=12):
+    seen = []
+
+    def check(res):
+        assert len(res.rows) == w.heads * w.n_query_blocks
         _check_step(res, w)
+        seen.append(res.position)
+
+    n_steps = 2 if topk == 16 else 1
+    Hn.run_stream(w, n_steps=n_steps, check_ring=(topk == 16), on_step=check)
+    assert len(seen) == n_steps
 
 
 def test_truncated_window_ragged_counts():
@@ -184,6 +209,39 @@ def test_programmatic_dependent_launch_matches_plain_launches():
         runs.append(outs)
     for (o1, k1, c1), (o2, k2, c2) in zip(*runs):
         assert torch.equal(k1, k2) and torch.equal(c1, c2) and torch.equal(o1, o2)
+
+
+def test_chained_draft_after_multi_layer_append_matches_plain_launches():
+    # A cold-start append of 3 block-layers, then a draft of only the newest
+    # layer launched as a programmatic dependent of that append: the draft must
+    # not read the key means of any of the 3 layers before the append completed
+    # (the cache records how many layers the append wrote).  Kept lists and
+    # scores equal those of plain launches bit for bit.
+    import dataclasses
+    L = _lib()
+    w = W.WORKLOADS["768x1280"]
+    dev = torch.device("cuda")
+    q3, k3, v3 = [t.to(dev) for t in W.gen_layers(w, 0, 3)]
+    q_new = q3[:, 4:6].contiguous()  # the newest layer's queries
+    runs = []
+    for chained in (True, False):
+        cache = L.KVCache.allocate(4, w.heads, w.grid_h, w.grid_w, dev)
+        st = torch.zeros((1,), dtype=torch.int32, device=dev)
+        p = L.make_params(w.heads, w.grid_h, w.grid_w, 1, w.topk, flags=L.LCSA_FLAG_PDL if chained else 0)
+        kept = torch.empty((w.heads, w.blocks_per_layer, w.topk), dtype=torch.int32, device=dev)
+        cnt = torch.empty((w.heads, w.blocks_per_layer), dtype=torch.int32, device=dev)
+        scores = torch.empty((w.heads, w.blocks_per_layer, 3 * w.blocks_per_layer), dtype=torch.float32,
+                             device=dev)
+        for _ in range(3):  # the same append and draft, repeated
+            cache.reset()
+            L.lcsa_cache_append(cache, k3, v3, d_status=st)
+            assert cache.desc.appended == 3 and cache.count == 3
+            L.lcsa_draft_mask(p, q_new, cache, kept, cnt, scores, d_status=st)
+        torch.cuda.synchronize()
+        assert st.item() == 0
+        runs.append((kept.clone(), cnt.clone(), scores.clone()))
+    for a, b in zip(*runs):
+        assert torch.equal(a, b)
 
 
 def test_host_stream_matches_direct_steps():

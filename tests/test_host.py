@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.lcsa_version() == 100
+    assert lib.lcsa_version() == 101
     assert L.status_string(L.LCSA_OK) == "LCSA_OK"
     assert L.status_string(L.LCSA_ERR_TIMEOUT) == "LCSA_ERR_TIMEOUT"
     assert L.status_string(L.LCSA_ERR_BAD_INDEX | L.LCSA_ERR_TIMEOUT).startswith("LCSA_ERR_TIMEOUT|")
@@ -65,6 +65,33 @@ def test_cache_append_rejects_bad_arguments_without_touching_the_gpu(lib):
     assert lib.lcsa_cache_append(ctypes.byref(bad), 0x40000, 0x50000, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
 
 
+def test_cache_appended_field_is_validated(lib):
+    # layers written by the last append: 0..capacity
+    z = ctypes.c_void_p(0x60000)
+    p = L.make_params(2, 4, 4, 1, 8)
+    for bad in (-1, 5):
+        c = _fake_cache(appended=bad)
+        assert lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None) == \
+            L.LCSA_ERR_INVALID_ARG
+        assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+
+
+# A call that passes validation goes on to launch a kernel: with the fake
+# pointers of these tests that must only happen where no GPU exists.
+no_gpu_only = pytest.mark.skipif(torch.cuda.is_available(),
+                                 reason="fake device pointers: runs only where the call cannot reach a GPU")
+
+
+@no_gpu_only
+def test_append_of_more_than_sixteen_layers_passes_validation(lib):
+    # the ring slots are computed on the device: any n_layers <= window is accepted
+    c = _fake_cache(capacity=40, window=40, count=0, heads=1)
+    rc = lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 33, 0, None, None)
+    assert rc != L.LCSA_ERR_INVALID_ARG
+    assert c.count == 0 and c.appended == 0  # nothing enqueued without a GPU: state unchanged
+
+
+@no_gpu_only
 def test_cache_window_and_overlap_rules(lib):
     k, v = 0x40000, 0x50000
     # at most `window` layers resident, window <= capacity
@@ -149,6 +176,53 @@ def test_bench_takes_max_over_two_gloo_ranks():
         assert abs(agg - 2 * 1e12 / 5e-3 / 1e12) < 1e-9
 
 
+def test_bench_gpus_must_match_world_size():
+    import bench
+    args = bench.parse_args(["--gpus", "2"])
+    with pytest.raises(SystemExit) as e:
+        bench.check_world(args, {"WORLD_SIZE": "1"})
+    assert "WORLD_SIZE=1" in str(e.value)
+    assert bench.check_world(args, {"WORLD_SIZE": "2"}) == "run"
+    # without torchrun, --gpus N > 1 starts N ranks itself
+    assert bench.check_world(args, {}) == "launch"
+    assert bench.check_world(bench.parse_args([]), {}) == "run"
+    # the reference arm runs once, on rank 0, whatever N is
+    assert bench.check_world(bench.parse_args(["--gpus", "4", "--impl", "reference"]), {}) == "run"
+    cmd = bench.launcher_argv(["--gpus", "2", "--steps", "5"], 2, 29500)
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert "--nproc-per-node=2" in cmd and cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-4:] == ["--gpus", "2", "--steps", "5"]
+
+
+def test_bench_main_exits_nonzero_on_world_mismatch():
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "8", "--steps", "1"],
+                       capture_output=True, text=True, timeout=300, cwd=root, env=env)
+    assert r.returncode != 0 and "WORLD_SIZE=1" in r.stderr
+
+
+def test_bench_config_is_shared_by_both_arms():
+    import bench
+    from diffusion_vsr_b200 import workloads as W
+    w = W.WORKLOADS["768x1408"]
+    kept = bench.chunk_kept_tiles(w)
+    assert kept == w.heads * w.n_query_blocks * w.topk == 15840
+    a = bench.bench_config(w, kept, 1)
+    for key in ("workload", "kv_len_layers", "local_range", "topk", "tflop_per_chunk", "l2", "parallelism"):
+        assert key in a
+    # ragged: a truncated 5-block window keeps fewer than topk at the edges
+    import dataclasses
+    wt = dataclasses.replace(W.WORKLOADS["768x1280"], local_mode=1, local_range=5, topk=40)
+    assert bench.chunk_kept_tiles(wt) < wt.heads * wt.n_query_blocks * wt.topk
+    # a reference step of n heads fits the run's budget
+    assert bench.reference_heads_per_step(w, 20, 5, 0.2) == 12
+    assert bench.reference_heads_per_step(w, 200, 10, 0.2) == 3
+    assert bench.reference_heads_per_step(w, 10000, 10, 5.0) == 1
+
+
 def test_reference_arm_prints_one_json_line():
     # `bench.py --impl reference` times the oracle (the pages ship no runnable
     # reference) and prints one JSON line with the contract's keys.
@@ -165,3 +239,7 @@ def test_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    import bench
+    from diffusion_vsr_b200 import workloads as W
+    w = W.WORKLOADS["tiny"]
+    assert d["config"] == bench.bench_config(w, bench.chunk_kept_tiles(w), 1)
