@@ -35,6 +35,12 @@ design notes):
   scores; the draft softmax is monotone and only computed for checks.
 * The attention scale is 1/sqrt(D), the same as the draft scale.
 * Intra-block token order is (t, y, x) row-major.
+* Segment-masked attention (the Stage-1 teacher of the reading notes'
+  关键设计 1): a packed sequence of segments, each one clip (a video, or an
+  image as a single-frame video), its tokens contiguous and in the clip's
+  (t, y, x) row-major order; the attention is dense within a segment and
+  there is none across segments (the block-diagonal mask of the alpha_ij
+  equation).  No causal rule applies in that stage.
 
 Parity: every function below is pinned by ``tests/test_oracle.py`` against
 closed forms, brute force and library routines; none is "parity unpinned".
@@ -238,6 +244,52 @@ def dense_block_causal_attention(q_tok: np.ndarray, k_tok: np.ndarray, v_tok: np
             p = np.exp(logits - logits.max(axis=1, keepdims=True))
             out[h, t] = (p @ v[h, vis]) / p.sum(axis=1, keepdims=True)
     return out.reshape(H, Tq, Y, X, D)
+
+
+# ------------------------------------------------------ segment-masked attention
+
+def segment_ids(clips: Sequence[Tuple[int, int, int]]) -> np.ndarray:
+    """Segment id of every token of a packed sequence of clips.
+
+    clips: (latent frames, token rows, token columns) per clip, in sequence
+    order; an image is a clip of one frame (reading notes, 关键设计 1: images
+    are single-frame videos).  Clip s contributes f*Y*X consecutive tokens of
+    id s.
+    """
+    return np.concatenate([np.full(f * y * x, s, dtype=np.int64) for s, (f, y, x) in enumerate(clips)])
+
+
+def segment_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seg: np.ndarray, scale: float,
+                      row_chunk: int = 128) -> Tuple[np.ndarray, np.ndarray]:
+    """Dense attention under the block-diagonal segment mask (关键设计 1):
+
+        alpha_ij = exp(q_i k_j^T * scale) 1[seg(i) = seg(j)]
+                   / sum_l exp(q_i k_l^T * scale) 1[seg(i) = seg(l)],
+        out_i = sum_j alpha_ij v_j.
+
+    q, k, v: [H, N, D] (any float dtype holding exact values; arithmetic in
+    fp64); seg: [N] segment id per token.  The query rows are taken
+    ``row_chunk`` at a time, each row's softmax over all N keys with the mask.
+    Returns out [H, N, D] and the natural-log denominator lse [H, N].
+    """
+    H, N, D = q.shape
+    seg = np.asarray(seg)
+    out = np.empty((H, N, D))
+    lse = np.empty((H, N))
+    for h in range(H):
+        kh = k[h].astype(np.float64)
+        vh = v[h].astype(np.float64)
+        for r0 in range(0, N, row_chunk):
+            qr = q[h, r0:r0 + row_chunk].astype(np.float64)
+            logits = (qr @ kh.T) * scale
+            same = seg[r0:r0 + row_chunk, None] == seg[None, :]
+            logits = np.where(same, logits, -np.inf)
+            m = logits.max(axis=1, keepdims=True)
+            p = np.exp(logits - m)
+            l = p.sum(axis=1, keepdims=True)
+            out[h, r0:r0 + row_chunk] = (p @ vh) / l
+            lse[h, r0:r0 + row_chunk] = (m + np.log(l))[:, 0]
+    return out, lse
 
 
 # -------------------------------------------------------------- KV cache model

@@ -357,6 +357,69 @@ def test_sparse_attention_matches_masked_dense_softmax():
         np.testing.assert_allclose(res["out_blocks"][0, i], ref, atol=1e-12)
 
 
+# -------------------------------------------------- segment-masked attention
+
+def test_segment_ids_follow_the_clips():
+    seg = O.segment_ids([(1, 2, 4), (3, 2, 4), (1, 4, 4)])
+    assert seg.size == 8 + 24 + 16
+    assert np.array_equal(np.bincount(seg), [8, 24, 16])
+    assert np.all(np.diff(seg) >= 0)
+
+
+def test_segment_attention_equals_library_sdpa_with_block_diagonal_mask():
+    rng = np.random.default_rng(31)
+    seg = O.segment_ids([(1, 4, 8), (2, 4, 8), (1, 2, 8)])
+    H, N, D = 2, seg.size, 16
+    q, k, v = (rng.standard_normal((H, N, D)) for _ in range(3))
+    out, lse = O.segment_attention(q, k, v, seg, 0.25, row_chunk=40)
+    mask = torch.from_numpy(seg[:, None] == seg[None, :])
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(k)[None], torch.from_numpy(v)[None], attn_mask=mask,
+        scale=0.25)[0].numpy()
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+    # lse: log-sum-exp of the row's logits over its own segment only
+    from scipy.special import logsumexp
+    for h, i in [(0, 0), (1, N - 1), (0, 40), (1, 100)]:
+        own = seg == seg[i]
+        np.testing.assert_allclose(lse[h, i], logsumexp(q[h, i] @ k[h, own].T * 0.25), atol=1e-12)
+
+
+def test_segment_attention_is_each_segment_alone():
+    # brute force: every segment attended on its own, without any mask
+    rng = np.random.default_rng(32)
+    clips = [(1, 4, 4), (3, 4, 4), (2, 2, 4)]
+    seg = O.segment_ids(clips)
+    H, N, D = 1, seg.size, 8
+    q, k, v = (rng.standard_normal((H, N, D)) for _ in range(3))
+    out, _ = O.segment_attention(q, k, v, seg, 0.5)
+    for s in range(len(clips)):
+        idx = np.nonzero(seg == s)[0]
+        logits = q[0, idx] @ k[0, idx].T * 0.5
+        p = np.exp(logits - logits.max(1, keepdims=True))
+        np.testing.assert_allclose(out[0, idx], p @ v[0, idx] / p.sum(1, keepdims=True), atol=1e-12)
+    # a token changing only another segment's keys/values does not move this segment's output
+    k2, v2 = k.copy(), v.copy()
+    other = seg == 1
+    k2[:, other] += 3.0
+    v2[:, other] -= 7.0
+    out2, _ = O.segment_attention(q, k2, v2, seg, 0.5)
+    np.testing.assert_allclose(out2[:, ~other], out[:, ~other], atol=1e-12)
+
+
+def test_one_segment_is_plain_dense_attention_and_constant_values_pass_through():
+    rng = np.random.default_rng(33)
+    H, N, D = 2, 64, 8
+    q, k = rng.standard_normal((H, N, D)), rng.standard_normal((H, N, D))
+    v = np.full((H, N, D), 2.5)
+    out, _ = O.segment_attention(q, k, v, np.zeros(N, dtype=int), 0.3)
+    np.testing.assert_allclose(out, 2.5, atol=1e-12)
+    v = rng.standard_normal((H, N, D))
+    out, _ = O.segment_attention(q, k, v, np.zeros(N, dtype=int), 0.3)
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(q), torch.from_numpy(k),
+                                                           torch.from_numpy(v), scale=0.3).numpy()
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+
+
 # ------------------------------------------------------------------ KV cache
 
 def test_cache_keeps_newest_layers_and_drops_oldest():
