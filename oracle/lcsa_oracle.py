@@ -35,6 +35,19 @@ design notes):
   scores; the draft softmax is monotone and only computed for checks.
 * The attention scale is 1/sqrt(D), the same as the draft scale.
 * Intra-block token order is (t, y, x) row-major.
+* Rotary position embedding (RoPE), which the reading notes name (背景,
+  关键设计 3) as the relative position code whose periodicity the local
+  window contains, with no layout: each adjacent pair of dimensions (2i,
+  2i+1) of q and k is rotated by the angle pos * w; the 64 pairs of a 128-dim
+  head are split into three axis bands over the token coordinates, time
+  (pairs 0-21), rows (22-42) and columns (43-63); inside a band of n pairs
+  w_i = base^(-i/n), base 10000; the time position is the absolute latent
+  frame index in the stream, the row/column positions the token row/column.
+  The rotated q and k are bf16 tensors (the attention's inputs): the rotation
+  is taken in the kernel's precision (fp32 cos/sin rounded from fp64, fp32
+  products and sum, one rounding each) and rounded to bf16 (nearest even),
+  because that rounding decides the bf16 values everything after is computed
+  from.
 * Segment-masked attention (the Stage-1 teacher of the reading notes'
   关键设计 1): a packed sequence of segments, each one clip (a video, or an
   image as a single-frame video), its tokens contiguous and in the clip's
@@ -246,6 +259,57 @@ def dense_block_causal_attention(q_tok: np.ndarray, k_tok: np.ndarray, v_tok: np
     return out.reshape(H, Tq, Y, X, D)
 
 
+# ------------------------------------------------------------------- RoPE
+
+ROPE_BANDS = (("t", 0, 22), ("y", 22, 21), ("x", 43, 21))  # (axis, first pair, pairs) of a 128-dim head
+
+
+def rope_angles(positions: np.ndarray, n_pairs: int, base: float) -> np.ndarray:
+    """Angles pos * w_i, w_i = base^(-i / n_pairs), i < n_pairs, in fp64: [len(positions), n_pairs]."""
+    w = np.power(float(base), -np.arange(n_pairs, dtype=np.float64) / n_pairs)
+    return np.asarray(positions, dtype=np.float64)[:, None] * w[None, :]
+
+
+def apply_rope(x_tok: np.ndarray, frame0: int, base: float, precision: str = "exact") -> np.ndarray:
+    """Rotate every dimension pair of a token-layout tensor [H, T, Y, X, 128].
+
+    Pair (2i, 2i+1) of the token at (frame t, row y, column x) turns by the
+    angle of its band's coordinate: (frame0 + t), y or x times w_i.
+    precision "exact": fp64 arithmetic, no rounding.  "kernel": cos and sin
+    rounded to fp32, a' = fl(fl(a cos) - fl(b sin)), b' = fl(fl(a sin) + fl(b cos))
+    in fp32, then rounded to bf16 (round to nearest even); returned as fp32
+    holding the bf16 values.
+    """
+    if precision not in ("exact", "kernel"):
+        raise ValueError(precision)
+    H, T, Y, X, D = x_tok.shape
+    if D != 128:
+        raise ValueError("the band layout is that of a 128-dim head")
+    pos = {"t": np.arange(T) + frame0, "y": np.arange(Y), "x": np.arange(X)}
+    shape = {"t": (1, T, 1, 1), "y": (1, 1, Y, 1), "x": (1, 1, 1, X)}
+    if precision == "exact":
+        out = np.array(x_tok, dtype=np.float64)
+    else:
+        out = np.array(x_tok, dtype=np.float32)
+    for axis, p0, n in ROPE_BANDS:
+        ang = rope_angles(pos[axis], n, base)  # [len, n]
+        c, s = np.cos(ang), np.sin(ang)
+        if precision == "kernel":
+            c, s = c.astype(np.float32), s.astype(np.float32)
+        for i in range(n):
+            d = 2 * (p0 + i)
+            ci = c[:, i].reshape(shape[axis])
+            si = s[:, i].reshape(shape[axis])
+            a = out[..., d].copy()
+            b = out[..., d + 1].copy()
+            out[..., d] = a * ci - b * si
+            out[..., d + 1] = a * si + b * ci
+    if precision == "kernel":
+        import torch
+        out = torch.from_numpy(out).to(torch.bfloat16).to(torch.float32).numpy()
+    return out
+
+
 # ------------------------------------------------------ segment-masked attention
 
 def segment_ids(clips: Sequence[Tuple[int, int, int]]) -> np.ndarray:
@@ -260,7 +324,7 @@ def segment_ids(clips: Sequence[Tuple[int, int, int]]) -> np.ndarray:
 
 
 def segment_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seg: np.ndarray, scale: float,
-                      row_chunk: int = 128) -> Tuple[np.ndarray, np.ndarray]:
+                      row_chunk: int = 128, query_rows: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
     """Dense attention under the block-diagonal segment mask (关键设计 1):
 
         alpha_ij = exp(q_i k_j^T * scale) 1[seg(i) = seg(j)]
@@ -270,19 +334,22 @@ def segment_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seg: np.ndarr
     q, k, v: [H, N, D] (any float dtype holding exact values; arithmetic in
     fp64); seg: [N] segment id per token.  The query rows are taken
     ``row_chunk`` at a time, each row's softmax over all N keys with the mask.
-    Returns out [H, N, D] and the natural-log denominator lse [H, N].
+    Returns out [H, N, D] and the natural-log denominator lse [H, N]; with
+    ``query_rows`` (token indices) only those rows: out [H, len, D], lse [H, len].
     """
     H, N, D = q.shape
     seg = np.asarray(seg)
-    out = np.empty((H, N, D))
-    lse = np.empty((H, N))
+    rows = np.arange(N) if query_rows is None else np.asarray(query_rows)
+    out = np.empty((H, rows.size, D))
+    lse = np.empty((H, rows.size))
     for h in range(H):
         kh = k[h].astype(np.float64)
         vh = v[h].astype(np.float64)
-        for r0 in range(0, N, row_chunk):
-            qr = q[h, r0:r0 + row_chunk].astype(np.float64)
+        for r0 in range(0, rows.size, row_chunk):
+            sel = rows[r0:r0 + row_chunk]
+            qr = q[h, sel].astype(np.float64)
             logits = (qr @ kh.T) * scale
-            same = seg[r0:r0 + row_chunk, None] == seg[None, :]
+            same = seg[sel, None] == seg[None, :]
             logits = np.where(same, logits, -np.inf)
             m = logits.max(axis=1, keepdims=True)
             p = np.exp(logits - m)

@@ -357,6 +357,81 @@ def test_sparse_attention_matches_masked_dense_softmax():
         np.testing.assert_allclose(res["out_blocks"][0, i], ref, atol=1e-12)
 
 
+# ------------------------------------------------------------------- RoPE
+
+def _placed(vec, T, Y, X, t, y, x):
+    z = np.zeros((1, T, Y, X, vec.size))
+    z[0, t, y, x] = vec
+    return z
+
+
+def test_rope_dot_products_depend_only_on_relative_position():
+    # q at (t1, y1, x1), k at (t2, y2, x2): moving both by the same offset along
+    # every axis (time through frame0, space inside a bigger grid) keeps q.k
+    rng = np.random.default_rng(41)
+    qv, kv = rng.standard_normal(128), rng.standard_normal(128)
+    T, Y, X = 4, 24, 24
+    for (t1, y1, x1), (t2, y2, x2), (dt, dy, dx) in [((0, 1, 2), (3, 5, 0), (7, 4, 9)),
+                                                    ((2, 0, 0), (0, 7, 7), (1000, 10, 3))]:
+        def dot(f0, oy, ox, q_only_y=0):
+            qy = y1 + oy + q_only_y
+            q = O.apply_rope(_placed(qv, T, Y, X, t1, qy, x1 + ox), f0, 10000.0)
+            k = O.apply_rope(_placed(kv, T, Y, X, t2, y2 + oy, x2 + ox), f0, 10000.0)
+            return float(q[0, t1, qy, x1 + ox] @ k[0, t2, y2 + oy, x2 + ox])
+        base = dot(5, 0, 0)
+        assert abs(dot(5 + dt, dy, dx) - base) < 1e-9 * (np.abs(qv).sum() * np.abs(kv).sum())
+        # moving the query alone changes it
+        assert abs(dot(5, 0, 0, q_only_y=1) - base) > 1e-6
+
+
+def test_rope_preserves_pair_norms_and_is_identity_at_the_origin():
+    rng = np.random.default_rng(42)
+    x = rng.standard_normal((2, 2, 8, 16, 128))
+    r = O.apply_rope(x, 11, 10000.0)
+    np.testing.assert_allclose(np.hypot(r[..., 0::2], r[..., 1::2]), np.hypot(x[..., 0::2], x[..., 1::2]),
+                               rtol=1e-12)
+    assert not np.allclose(r, x)
+    # frame 0, row 0, column 0: every angle is 0
+    np.testing.assert_array_equal(O.apply_rope(x, 0, 10000.0)[:, 0, 0, 0], x[:, 0, 0, 0])
+    xb = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+    np.testing.assert_array_equal(O.apply_rope(xb, 0, 10000.0, "kernel")[:, 0, 0, 0], xb[:, 0, 0, 0])
+
+
+def test_rope_pair_is_a_complex_multiplication_with_the_band_frequencies():
+    # closed forms of the band layout: 22 + 21 + 21 pairs; inside a band the
+    # first pair turns by the position itself and the frequencies fall
+    # geometrically by base^(-1/n) down to base^(-(n-1)/n)
+    assert [n for _, _, n in O.ROPE_BANDS] == [22, 21, 21]
+    assert [p0 for _, p0, _ in O.ROPE_BANDS] == [0, 22, 43]
+    rng = np.random.default_rng(43)
+    x = rng.standard_normal((1, 3, 8, 8, 128))
+    f0, base = 4, 10000.0
+    r = O.apply_rope(x, f0, base)
+    t, y, xx = 2, 5, 3
+    pos = {"t": f0 + t, "y": y, "x": xx}
+    for axis, p0, n in O.ROPE_BANDS:
+        for i in (0, 1, n - 1):
+            w = 1.0 if i == 0 else (base ** (-1.0 / n)) ** i
+            z = complex(x[0, t, y, xx, 2 * (p0 + i)], x[0, t, y, xx, 2 * (p0 + i) + 1]) * np.exp(1j * pos[axis] * w)
+            assert abs(r[0, t, y, xx, 2 * (p0 + i)] - z.real) < 1e-9
+            assert abs(r[0, t, y, xx, 2 * (p0 + i) + 1] - z.imag) < 1e-9
+
+
+def test_rope_kernel_precision_is_the_exact_rotation_rounded_to_bf16():
+    rng = np.random.default_rng(44)
+    x = torch.from_numpy(rng.standard_normal((1, 2, 8, 16, 128)).astype(np.float32)).to(torch.bfloat16)
+    xf = x.to(torch.float32).numpy()
+    exact = O.apply_rope(xf, 9, 10000.0)
+    kern = O.apply_rope(xf, 9, 10000.0, "kernel")
+    # bf16 values (8 significant bits): within half a bf16 ulp of the exact
+    # rotation, plus the fp32 arithmetic before the rounding
+    assert np.array_equal(torch.from_numpy(kern).to(torch.bfloat16).to(torch.float32).numpy(), kern)
+    tol = np.abs(exact) * 2.0 ** -8 + 1e-6
+    assert np.all(np.abs(kern - exact) <= tol)
+    with pytest.raises(ValueError):
+        O.apply_rope(xf, 0, 10000.0, "bogus")
+
+
 # -------------------------------------------------- segment-masked attention
 
 def test_segment_ids_follow_the_clips():
@@ -377,6 +452,11 @@ def test_segment_attention_equals_library_sdpa_with_block_diagonal_mask():
         torch.from_numpy(q)[None], torch.from_numpy(k)[None], torch.from_numpy(v)[None], attn_mask=mask,
         scale=0.25)[0].numpy()
     np.testing.assert_allclose(out, ref, atol=1e-12)
+    # a subset of query rows gives those rows of the full result
+    rows = np.array([0, 5, 47, 63, 64, 100, N - 1])
+    o_sub, l_sub = O.segment_attention(q, k, v, seg, 0.25, row_chunk=3, query_rows=rows)
+    np.testing.assert_allclose(o_sub, out[:, rows], atol=1e-12)
+    np.testing.assert_allclose(l_sub, lse[:, rows], atol=1e-12)
     # lse: log-sum-exp of the row's logits over its own segment only
     from scipy.special import logsumexp
     for h, i in [(0, 0), (1, N - 1), (0, 40), (1, 100)]:
