@@ -37,6 +37,8 @@
 //                  it with two TMA stores into token layout (the reverse
 //                  partition); the other group hands over its (m, l) through
 //                  shared memory and starts the next row at once.
+//   warp 3         with RoPE only: rotates each Q tile in place once it has
+//                  landed; the MMA issuers wait for the rotated tile.
 // TMEM (512 columns): S_w at 128*w, O_w at 256 + 128*w.
 // Launched as a programmatic dependent of the draft mask (LCSA_FLAG_PDL), the
 // set-up overlaps the draft's tail and the producer waits for it before it
@@ -46,6 +48,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "rope.cuh"
 #include "../../include/lcsa.h"
 
 namespace lcsa {
@@ -73,6 +76,7 @@ struct __align__(1024) AttnSmem {
     uint8_t k[kKStages][kTileBytes];
     uint8_t v[kVStages][kTileBytes];
     uint64_t bar_qfull[2];
+    uint64_t bar_qrot[2];   // with RoPE: the Q tile of the buffer is rotated (warp 3)
     uint64_t bar_qempty[2];
     uint64_t bar_kfull[kKStages];
     uint64_t bar_kempty[kKStages];
@@ -213,10 +217,12 @@ __device__ __forceinline__ bool issue_pv(AttnSmem &sm, const MmaCtx &m, int w, i
     return true;
 }
 
+// kRope: the Q tiles are rotated by warp 3 (RoPE) before the MMAs read them.
+template <bool kRope>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                     const AttnArgs a, uint16_t *__restrict__ out) {
+                     const AttnArgs a, const AttnRope rope, uint16_t *__restrict__ out) {
     extern __shared__ uint8_t smem_raw[];
     AttnSmem &sm = *reinterpret_cast<AttnSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                   ~static_cast<uintptr_t>(1023));
@@ -228,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&sm.bar_qfull[b]), 1);
+            mbar_init(smem_u32(&sm.bar_qrot[b]), 1);
             mbar_init(smem_u32(&sm.bar_qempty[b]), 1);  // the late group's output copy read the buffer
             mbar_init(smem_u32(&sm.bar_sfull[b]), 1);
             for (int qq = 0; qq < 4; ++qq) mbar_init(smem_u32(&sm.bar_pq[qq][b]), 4);  // one arrival per warp
@@ -248,7 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(smem_u32(&sm.bar_mlfree), 4);   // the late group's warps
         for (int i = 0; i < kInfoSlots; ++i) {
             mbar_init(smem_u32(&sm.bar_info_full[i]), 1);
-            mbar_init(smem_u32(&sm.bar_info_empty[i]), 10);  // 2 MMA issuers + 8 softmax warps
+            // 2 MMA issuers + 8 softmax warps (+ the rotation warp)
+            mbar_init(smem_u32(&sm.bar_info_empty[i]), kRope ? 11 : 10);
         }
         sm.abort_word = 0;
         fence_mbar_init();
@@ -391,7 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (n == 0) continue;
                 const int qb = act & 1;
                 const int n_mine = (n - w + 1) >> 1;
-                ok = mbar_wait(smem_u32(&sm.bar_qfull[qb]), (act >> 1) & 1, abort_word, to);
+                // the Q tile has landed (and, with RoPE, been rotated by warp 3)
+                ok = mbar_wait(smem_u32(kRope ? &sm.bar_qrot[qb] : &sm.bar_qfull[qb]), (act >> 1) & 1, abort_word,
+                               to);
                 // Tile w + 2i of the row follows tile w + 2i - 1 of the other group
                 // (for group 0's first tile: the previous row's last tile, when
                 // that row had an even count).
@@ -422,6 +432,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Every MMA issued must be complete before TMEM is freed.
             mma_commit(smem_u32(&sm.bar_drain[w]));
             mbar_wait_drain(smem_u32(&sm.bar_drain[w]), 0, to);
+        }
+        __syncwarp();
+    } else if (warp == 3) {
+        // ------------------------------------------------- Q rotation (RoPE)
+        // Lane l rotates pairs l (dims 2l, 2l+1, first 16 KB half of the Q tile)
+        // and l + 32 (same place in the second half) of all 128 tokens, in place
+        // in the 128-byte swizzled tile: token n's 16-byte chunk c sits at chunk
+        // position c ^ (n & 7).  Pair l turns with the frame (l < 22) or the token
+        // row; pair l + 32 with the token row (l < 11) or the token column.  (cos,
+        // sin) are evaluated (fp64, rounded to fp32) per frame, row or column as
+        // the rows of the tile are walked: few registers, as this warp runs with
+        // the control warpgroup's budget.
+        if (kRope) {
+            const int p0 = lane, p1 = lane + 32;
+            const int ax0 = rope_axis(p0), ax1 = rope_axis(p1);
+            const double w0 = rope_freq(p0, rope.base), w1 = rope_freq(p1, rope.base);
+            const uint32_t word = static_cast<uint32_t>(((lane >> 2) << 4) + (lane & 3) * 4);  // chunk, word
+            int act = 0, r = 0;
+            bool ok = true;
+            for (int unit = blockIdx.x; unit < a.n_units; unit += gridDim.x, ++r) {
+                const int is = r % kInfoSlots;
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(smem_u32(&sm.bar_info_full[is]), (r / kInfoSlots) & 1, abort_word, to));
+                if (!ok) break;
+                const int n = *reinterpret_cast<volatile int32_t *>(&sm.info_n[is]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sm.bar_info_empty[is]));
+                if (n == 0) continue;
+                const int qb = act & 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_qfull[qb]), (act >> 1) & 1, abort_word, to));
+                if (!ok) break;
+                const RowGeom rg = row_geom(a, unit);
+                // column-band angles of pair l + 32 for the block's 8 token columns
+                float2 cx[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) cx[x] = rope_cs(rg.qbx * 8 + x, w1);
+                uint8_t *tile = sm.q[qb];
+#pragma unroll 1
+                for (int ty = 0; ty < 16; ++ty) {  // frame ty / 8, token row ty % 8 of the block
+                    const int t = ty >> 3, y = ty & 7;
+                    const float2 v0 = rope_cs(ax0 == 0 ? rope.frame0 + 2 * rg.ql + t : rg.qby * 8 + y, w0);
+                    const float2 vy = rope_cs(rg.qby * 8 + y, w1);
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) {
+                        const int tok = 8 * ty + x;
+                        uint32_t *w_lo = reinterpret_cast<uint32_t *>(tile + tok * 128 + (word ^ (x << 4)));
+                        uint32_t *w_hi = reinterpret_cast<uint32_t *>(tile + kHalfBytes + tok * 128 + (word ^ (x << 4)));
+                        const float2 v1 = ax1 == 1 ? vy : cx[x];
+                        *w_lo = rope_rotate(*w_lo, v0.x, v0.y);
+                        *w_hi = rope_rotate(*w_hi, v1.x, v1.y);
+                    }
+                }
+                fence_proxy_async_smem();  // the MMAs read the tile through the async proxy
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sm.bar_qrot[qb]));
+                ++act;
+            }
         }
         __syncwarp();
     } else if (warp >= kSoftmaxWarp0) {
@@ -704,15 +771,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                             const CUtensorMap &tm_o, const AttnArgs &a, bool pdl, void *out, const DeviceInfo &dev,
-                             cudaStream_t stream) {
-    static std::atomic<int> smem_set[kMaxDevices];
+                             const CUtensorMap &tm_o, const AttnArgs &a, const AttnRope &rope, bool pdl, void *out,
+                             const DeviceInfo &dev, cudaStream_t stream) {
+    static std::atomic<int> smem_set[2][kMaxDevices];
     const size_t smem = sizeof(AttnSmem) + 1024;
-    const cudaError_t e = ensure_smem_limit(attention_kernel, dev.device, smem, smem_set);
+    const bool rot = rope.base != 0.f;
+    const cudaError_t e = rot ? ensure_smem_limit(attention_kernel<true>, dev.device, smem, smem_set[1])
+                              : ensure_smem_limit(attention_kernel<false>, dev.device, smem, smem_set[0]);
     if (e != cudaSuccess) return e;
     const int grid = a.n_units < dev.sms ? a.n_units : dev.sms;
-    return launch_kernel(attention_kernel, dim3(grid), dim3(kThreads), smem, stream, pdl, tm_q, tm_k, tm_v, tm_o, a,
-                         static_cast<uint16_t *>(out));
+    if (rot)
+        return launch_kernel(attention_kernel<true>, dim3(grid), dim3(kThreads), smem, stream, pdl, tm_q, tm_k, tm_v,
+                             tm_o, a, rope, static_cast<uint16_t *>(out));
+    return launch_kernel(attention_kernel<false>, dim3(grid), dim3(kThreads), smem, stream, pdl, tm_q, tm_k, tm_v, tm_o,
+                         a, rope, static_cast<uint16_t *>(out));
 }
 
 }  // namespace lcsa

@@ -23,6 +23,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "rope.cuh"
 #include "../../include/lcsa.h"
 
 namespace lcsa {
@@ -99,6 +100,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int pr = tid & 63;   // dimensions 2 pr, 2 pr + 1
     const int half = tid >> 6;  // tokens [64 half, 64 half + 64)
+    const bool rope = a.rope_base != 0.f;
+    const int rope_axis_pr = rope_axis(pr);
+    const double rope_w = rope ? rope_freq(pr, a.rope_base) : 0.0;
+    // (cos, sin) of pos * w and of w, for the angle-addition steps along a row or column
+    double step_c = 1.0, step_s = 0.0;
+    if (rope && rope_axis_pr != 0) rope_sincos(rope_w, step_s, step_c);
     bool ok = true;
     for (int i = 0; i < n_mine; ++i) {
         const int s = i % kStages;
@@ -112,6 +119,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         int slot = a.first_slot + un.li;  // < 2 * capacity
         if (slot >= a.capacity) slot -= a.capacity;
         const size_t blk = (static_cast<size_t>(slot) * a.heads + un.h) * a.nblk + un.b;
+        if (rope) {
+            // Pair pr of this thread's 64 tokens (frame `half` of the block), rotated
+            // in place.  cs[i]: the angle of the i-th row (row band) or column (column
+            // band) of the block, or of the frame (time band: every entry), from one
+            // fp64 sincos and exact angle-addition steps in fp64.
+            const int by = mul_div(un.b, a.m_gw), bx = un.b - by * a.grid_w;
+            const int pos0 = rope_axis_pr == 0 ? a.rope_frame0 + 2 * un.li + half
+                                               : (rope_axis_pr == 1 ? by * 8 : bx * 8);
+            double c, sn;
+            rope_sincos(static_cast<double>(pos0) * rope_w, sn, c);
+            float2 cs[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                cs[i] = make_float2(__double2float_rn(c), __double2float_rn(sn));
+                const double c2 = c * step_c - sn * step_s;
+                sn = sn * step_c + c * step_s;
+                c = c2;
+            }
+            uint32_t *kw_rw = reinterpret_cast<uint32_t *>(sm.k[s]) + half * 64 * (kHeadDim / 2) + pr;
+#pragma unroll
+            for (int yy = 0; yy < 8; ++yy) {
+#pragma unroll
+                for (int xx = 0; xx < 8; ++xx) {
+                    const float2 v = rope_axis_pr == 2 ? cs[xx] : cs[yy];  // (time band: all equal)
+                    uint32_t *p = kw_rw + (8 * yy + xx) * (kHeadDim / 2);
+                    *p = rope_rotate(*p, v.x, v.y);
+                }
+            }
+            fence_proxy_async_smem();  // the rotated tile is read by the bulk store (async proxy)
+            __syncthreads();           // every pair of the tile is rotated before the means read it
+        }
         // k mean: this thread sums its 64 tokens of two dimensions
         const uint32_t *kw = reinterpret_cast<const uint32_t *>(sm.k[s]) + half * 64 * (kHeadDim / 2) + pr;
         float lo = 0.f, hi = 0.f;

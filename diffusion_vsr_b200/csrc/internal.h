@@ -85,32 +85,57 @@ struct AttnArgs {
     uint64_t m_nq, m_nblk, m_gw;
 };
 
+// Rotation of the Q tiles (a separate kernel argument: the kernel instance
+// without rotation ignores it).
+struct AttnRope {
+    float base;            // 0: no rotation
+    int32_t frame0;        // stream position of q's first frame
+};
+
 // Multiplier of the exact multiply-high division by d (1 <= d).
 inline uint64_t div_magic_host(uint32_t d) { return ((1ull << 32) + d - 1) / d; }
 
 cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                             const CUtensorMap &tm_o, const AttnArgs &a, bool pdl, void *out, const DeviceInfo &dev,
-                             cudaStream_t stream);
+                             const CUtensorMap &tm_o, const AttnArgs &a, const AttnRope &rope, bool pdl, void *out,
+                             const DeviceInfo &dev, cudaStream_t stream);
 
-// Draft mask: q block means, scores over allowed candidates, top-k.
+// Draft mask: q block means, scores over allowed candidates, top-k.  One CTA
+// per tile of tile_h x tile_w query blocks of one (head, query layer); rmax
+// (>= tile rows, one of 4, 8, 12, 16) and kpt (union keys per thread and
+// round, 1..3) select the kernel instance.
 struct DraftArgs {
-    const uint16_t *q;     // bf16 token layout
     const float *kmean;    // [cap][H][nblk][128]
-    int32_t heads, grid_h, grid_w, nblk, q_layers, tq, tok_h, tok_w;
+    int32_t heads, grid_h, grid_w, nblk, q_layers;
     int32_t capacity, oldest, count;
-    int32_t fresh_layers;  // newest layers the preceding kernel may still be writing (PDL)
     int32_t local_range, local_mode, topk;
     int32_t cand_cap;      // most allowed candidates of a row, rounded up to 32
-    uint64_t m_nq, m_nblk, m_gw;  // multiply-high multipliers of q_layers*nblk, nblk, grid_w
+    int32_t tile_h, tile_w, tiles_y, tiles_x;
+    int32_t rmax, kpt;
+    // ceil(2^32 / d) for d = tiles_y * tiles_x, q_layers, tiles_x: n / d = (n * m) >> 32
+    uint64_t m_tiles, m_ql, m_tiles_x;
     float scale;
     int32_t *kept_idx;
     int32_t *kept_cnt;
     float *scores;         // may be null
     float *qmean;          // may be null
-    int32_t *status;
+    int32_t *status;       // may be null
+    uint64_t timeout_ns;
+    float rope_base;       // 0: no rotation of q
+    int32_t rope_frame0;   // stream position of q's first frame
+    int32_t rope_entries;  // rotation table entries of a tile (0 without rotation)
 };
 
-cudaError_t launch_draft(const DraftArgs &a, bool pdl, const DeviceInfo &dev, cudaStream_t stream);
+// Entries of a draft CTA's rotation table for tiles of tile_h x tile_w blocks.
+inline int draft_rope_entries(int tile_h, int tile_w) { return 2 * 22 + 8 * (tile_h + tile_w) * 21; }
+
+// Shared memory of the draft kernel instance (rmax, kpt) for rows of at most
+// cand_cap candidates, alignment slack included (0 for an unknown instance).
+size_t draft_smem_bytes(int rmax, int kpt, int cand_cap, int rope_entries);
+
+// tm_q: rank-4 map over q in token layout with a whole-block box (128 dims,
+// 8, 8, 2 frames), no swizzle.
+cudaError_t launch_draft(const CUtensorMap &tm_q, const DraftArgs &a, bool pdl, const DeviceInfo &dev,
+                         cudaStream_t stream);
 
 // Cache append: token layout -> block layout ring slots + k block means.
 struct AppendArgs {
@@ -123,11 +148,25 @@ struct AppendArgs {
     int32_t *status;                 // may be null
     uint64_t timeout_ns;
     int32_t flags;
+    float rope_base;                 // 0: no rotation of k
+    int32_t rope_frame0;             // stream position of the chunk's first frame
 };
 
 // tm_k / tm_v: rank-4 maps over the chunk's k / v in token layout with a
 // (128 dims, 8, 8, 2 frames) box, no swizzle (one box = one block, in block order).
 cudaError_t launch_cache_append(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const AppendArgs &a, bool pdl,
                                 const DeviceInfo &dev, cudaStream_t stream);
+
+// Kept lists of segment-masked dense attention: query tile i of segment s
+// keeps key tiles start[s] .. start[s + 1] - 1.
+constexpr int kMaxSegments = 256;
+struct SegmentArgs {
+    int32_t heads, tiles, topk, n_seg;
+    int32_t start[kMaxSegments + 1];  // first tile of every segment, then the tile count
+    int32_t *kept_idx;
+    int32_t *kept_cnt;
+};
+
+cudaError_t launch_segment_mask(const SegmentArgs &a, cudaStream_t stream);
 
 }  // namespace lcsa

@@ -26,23 +26,28 @@ LCSA_ERR_BAD_INDEX = 8
 LCSA_FLAG_FORCE_TIMEOUT = 1
 LCSA_FLAG_PDL = 2
 LCSA_MAX_CANDIDATES = 4096
+LCSA_MAX_SEGMENTS = 256
 
-EXPORTED_SYMBOLS = ("lcsa_cache_append", "lcsa_draft_mask", "lcsa_attention", "lcsa_status_string",
-                    "lcsa_version")
+EXPORTED_SYMBOLS = ("lcsa_cache_append", "lcsa_draft_mask", "lcsa_attention", "lcsa_segment_mask",
+                    "lcsa_status_string", "lcsa_version")
+
+
+class lcsa_rope(ctypes.Structure):
+    _fields_ = [("base", ctypes.c_float), ("frame0", ctypes.c_int32)]
 
 
 class lcsa_params(ctypes.Structure):
     _fields_ = [("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("grid_h", ctypes.c_int32),
                 ("grid_w", ctypes.c_int32), ("q_layers", ctypes.c_int32), ("local_range", ctypes.c_int32),
                 ("local_mode", ctypes.c_int32), ("topk", ctypes.c_int32), ("scale", ctypes.c_float),
-                ("flags", ctypes.c_int32)]
+                ("flags", ctypes.c_int32), ("rope", lcsa_rope)]
 
 
 class lcsa_kv_cache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("kmean", ctypes.c_void_p),
                 ("capacity", ctypes.c_int32), ("oldest", ctypes.c_int32), ("count", ctypes.c_int32),
                 ("heads", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
-                ("window", ctypes.c_int32), ("appended", ctypes.c_int32)]
+                ("window", ctypes.c_int32)]
 
 
 class LcsaError(RuntimeError):
@@ -66,12 +71,15 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     P = ctypes.POINTER
     vp = ctypes.c_void_p
-    lib.lcsa_cache_append.argtypes = [P(lcsa_kv_cache), vp, vp, ctypes.c_int32, ctypes.c_int32, vp, vp]
+    lib.lcsa_cache_append.argtypes = [P(lcsa_kv_cache), vp, vp, ctypes.c_int32, ctypes.c_int32, P(lcsa_rope), vp,
+                                      vp]
     lib.lcsa_cache_append.restype = ctypes.c_int
     lib.lcsa_draft_mask.argtypes = [P(lcsa_params), vp, P(lcsa_kv_cache), vp, vp, vp, vp, vp, vp]
     lib.lcsa_draft_mask.restype = ctypes.c_int
     lib.lcsa_attention.argtypes = [P(lcsa_params), vp, P(lcsa_kv_cache), vp, vp, vp, vp, vp, vp]
     lib.lcsa_attention.restype = ctypes.c_int
+    lib.lcsa_segment_mask.argtypes = [P(ctypes.c_int32), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp, vp, vp]
+    lib.lcsa_segment_mask.restype = ctypes.c_int
     lib.lcsa_status_string.argtypes = [ctypes.c_int]
     lib.lcsa_status_string.restype = ctypes.c_char_p
     lib.lcsa_version.argtypes = []
@@ -106,8 +114,10 @@ def _check(fn: str, rc: int) -> None:
 
 
 def make_params(heads: int, grid_h: int, grid_w: int, q_layers: int, topk: int, local_range: int = 11,
-                local_mode: int = 0, scale: float = 0.0, flags: int = 0) -> lcsa_params:
-    return lcsa_params(heads, 128, grid_h, grid_w, q_layers, local_range, local_mode, topk, scale, flags)
+                local_mode: int = 0, scale: float = 0.0, flags: int = 0, rope_base: float = 0.0,
+                rope_frame0: int = 0) -> lcsa_params:
+    return lcsa_params(heads, 128, grid_h, grid_w, q_layers, local_range, local_mode, topk, scale, flags,
+                       lcsa_rope(rope_base, rope_frame0))
 
 
 @dataclass
@@ -144,15 +154,16 @@ class KVCache:
     def reset(self) -> None:
         self.desc.oldest = 0
         self.desc.count = 0
-        self.desc.appended = 0
 
 
 def lcsa_cache_append(cache: KVCache, k_tok: torch.Tensor, v_tok: torch.Tensor, n_layers: Optional[int] = None,
-                      d_status: Optional[torch.Tensor] = None, stream=None, flags: int = 0) -> None:
+                      d_status: Optional[torch.Tensor] = None, stream=None, flags: int = 0,
+                      rope: Optional[lcsa_rope] = None) -> None:
     if n_layers is None:
         n_layers = k_tok.shape[1] // 2
     rc = load_library().lcsa_cache_append(ctypes.byref(cache.desc), _ptr(k_tok), _ptr(v_tok), n_layers, flags,
-                                          _ptr(d_status), _stream(stream))
+                                          ctypes.byref(rope) if rope is not None else None, _ptr(d_status),
+                                          _stream(stream))
     _check("lcsa_cache_append", rc)
 
 
@@ -175,6 +186,49 @@ def lcsa_attention(params: lcsa_params, q_tok: torch.Tensor, cache: KVCache, kep
     _check("lcsa_attention", rc)
 
 
+def lcsa_segment_mask(seg_tiles, heads: int, kept_idx: torch.Tensor, kept_cnt: torch.Tensor,
+                      stream=None) -> None:
+    """Kept lists of segment-masked dense attention; ``seg_tiles`` is a host sequence."""
+    n = len(seg_tiles)
+    arr = (ctypes.c_int32 * max(n, 1))(*seg_tiles)
+    rc = load_library().lcsa_segment_mask(arr, n, heads, kept_idx.shape[-1], _ptr(kept_idx), _ptr(kept_cnt),
+                                          _stream(stream))
+    _check("lcsa_segment_mask", rc)
+
+
+class SegmentAttention:
+    """Segment-masked dense attention over a packed sequence of clips.
+
+    The Stage-1 teacher's attention (every token attends to its own segment
+    only) as three library calls: the packed k/v appended as one block-layer
+    per 128-token tile to a ring of grid 1 x 1, the kept lists of the segment
+    table, and the block-sparse attention over them.  q, k, v, out: bf16
+    [heads, 128 * tiles, 128] on the GPU, every segment a whole number of tiles.
+    """
+
+    def __init__(self, heads: int, seg_tiles, device="cuda"):
+        self.seg_tiles = [int(t) for t in seg_tiles]
+        self.tiles = sum(self.seg_tiles)
+        self.topk = max(self.seg_tiles)
+        self.heads = heads
+        self.cache = KVCache.allocate(self.tiles, heads, 1, 1, device)
+        self.params = make_params(heads, 1, 1, self.tiles, self.topk, local_range=0)
+        self.kept_idx = torch.empty((heads, self.tiles, self.topk), dtype=torch.int32, device=device)
+        self.kept_cnt = torch.empty((heads, self.tiles), dtype=torch.int32, device=device)
+        self.status = torch.zeros((1,), dtype=torch.int32, device=device)
+        lcsa_segment_mask(self.seg_tiles, heads, self.kept_idx, self.kept_cnt)
+
+    def run(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+            lse: Optional[torch.Tensor] = None) -> None:
+        shape = (self.heads, 128 * self.tiles, 128)
+        for t in (q, k, v, out):
+            if tuple(t.shape) != shape:
+                raise ValueError(f"expected {shape}, got {tuple(t.shape)}")
+        self.cache.reset()
+        lcsa_cache_append(self.cache, k, v, n_layers=self.tiles, d_status=self.status)
+        lcsa_attention(self.params, q, self.cache, self.kept_idx, self.kept_cnt, out, lse, d_status=self.status)
+
+
 class LcsaLayer:
     """One LCSA attention layer of a streaming DiT: cache + draft + attention.
 
@@ -184,12 +238,13 @@ class LcsaLayer:
     """
 
     def __init__(self, heads: int, grid_h: int, grid_w: int, q_layers: int, kv_len: int, topk: int,
-                 local_range: int = 11, local_mode: int = 0, device="cuda"):
-        self.params = make_params(heads, grid_h, grid_w, q_layers, topk, local_range, local_mode)
+                 local_range: int = 11, local_mode: int = 0, device="cuda", rope_base: float = 0.0):
+        self.params = make_params(heads, grid_h, grid_w, q_layers, topk, local_range, local_mode,
+                                  rope_base=rope_base)
         # step(): the draft follows the append and the attention the draft, neither of
         # which writes q or the output, so both may launch as programmatic dependents
         self.params_chained = make_params(heads, grid_h, grid_w, q_layers, topk, local_range, local_mode,
-                                          flags=LCSA_FLAG_PDL)
+                                          flags=LCSA_FLAG_PDL, rope_base=rope_base)
         # kv_len + q_layers resident layers plus q_layers spare slots: a step's append
         # never overwrites a layer the previous step reads (see step(overlap_previous))
         self.cache = KVCache.allocate(kv_len + 2 * q_layers, heads, grid_h, grid_w, device,
@@ -198,9 +253,15 @@ class LcsaLayer:
         self.kept_idx = torch.empty((heads, nq, topk), dtype=torch.int32, device=device)
         self.kept_cnt = torch.empty((heads, nq), dtype=torch.int32, device=device)
         self.status = torch.zeros((1,), dtype=torch.int32, device=device)
+        self.rope_base = rope_base
+        self.frame = 0  # stream position of the next appended frame (RoPE time axis)
+
+    def _rope(self, frame0: int) -> Optional[lcsa_rope]:
+        return lcsa_rope(self.rope_base, frame0) if self.rope_base else None
 
     def append(self, k_tok: torch.Tensor, v_tok: torch.Tensor) -> None:
-        lcsa_cache_append(self.cache, k_tok, v_tok, d_status=self.status)
+        lcsa_cache_append(self.cache, k_tok, v_tok, d_status=self.status, rope=self._rope(self.frame))
+        self.frame += k_tok.shape[1]
 
     def step(self, q_tok: torch.Tensor, k_tok: torch.Tensor, v_tok: torch.Tensor, out_tok: torch.Tensor,
              lse: Optional[torch.Tensor] = None, overlap_previous: bool = False) -> None:
@@ -211,8 +272,12 @@ class LcsaLayer:
         the append is then launched as its programmatic dependent and runs in the
         SMs that attention's last CTAs leave idle.
         """
+        frame0 = self.frame
         lcsa_cache_append(self.cache, k_tok, v_tok, d_status=self.status,
-                          flags=LCSA_FLAG_PDL if overlap_previous else 0)
+                          flags=LCSA_FLAG_PDL if overlap_previous else 0, rope=self._rope(frame0))
+        self.frame += k_tok.shape[1]
+        self.params.rope.frame0 = frame0
+        self.params_chained.rope.frame0 = frame0
         lcsa_draft_mask(self.params_chained, q_tok, self.cache, self.kept_idx, self.kept_cnt, d_status=self.status)
         lcsa_attention(self.params_chained, q_tok, self.cache, self.kept_idx, self.kept_cnt, out_tok, lse,
                        d_status=self.status)

@@ -195,6 +195,64 @@ def stream_plan(w: Workload):
     return prefill, steps
 
 
+# ------------------------------------------- segment-masked attention workloads
+
+@dataclasses.dataclass(frozen=True)
+class SegmentWorkload:
+    """A packed sequence of clips for the segment-masked attention of the
+    Stage-1 teacher (reading notes, 关键设计 1): images are clips of one latent
+    frame, videos clips of several; every clip is one segment, its tokens
+    contiguous in (t, y, x) row-major order.  Every clip must hold a whole
+    number of 128-token tiles."""
+    name: str
+    heads: int
+    clips: tuple            # ((latent frames, token rows, token columns), ...)
+    seed: int
+    head_dim: int = HEAD_DIM
+
+    @property
+    def seg_tokens(self):
+        return [f * y * x for f, y, x in self.clips]
+
+    @property
+    def seg_tiles(self):
+        tiles = []
+        for n in self.seg_tokens:
+            if n % BLOCK_TOKENS:
+                raise ValueError(f"{self.name}: a clip of {n} tokens is not a whole number of 128-token tiles")
+            tiles.append(n // BLOCK_TOKENS)
+        return tiles
+
+    @property
+    def tokens(self) -> int:
+        return sum(self.seg_tokens)
+
+    @property
+    def kept_tiles(self) -> int:
+        """Tiles the masked attention computes: every (query tile, key tile) pair of a segment."""
+        return self.heads * sum(t * t for t in self.seg_tiles)
+
+
+SEGMENT_WORKLOADS = {
+    # 256x512 px frames: 16 x 32 tokens = 4 tiles per latent frame
+    "small": SegmentWorkload("small", heads=2, clips=((1, 16, 32), (3, 16, 32), (1, 16, 32), (2, 16, 32)), seed=5),
+    # 768x1280 px frames (48 x 80 tokens = 30 tiles per latent frame): an image, a
+    # 5-latent-frame video, an image, a 3-latent-frame video
+    "768x1280": SegmentWorkload("768x1280", heads=12,
+                                clips=((1, 48, 80), (5, 48, 80), (1, 48, 80), (3, 48, 80)), seed=6),
+}
+
+
+def gen_segments(w: SegmentWorkload) -> List[torch.Tensor]:
+    """q, k, v of a packed segment sequence: bf16 CPU tensors [heads, tokens, head_dim],
+    i.i.d. N(0,1) drawn in fp32 from ``default_rng([seed * 1000, stream])`` and rounded RNE."""
+    out = []
+    for stream in (STREAM_Q, STREAM_K, STREAM_V):
+        x = _normal_f32(_rng(w.seed, 0, stream), (w.heads, w.tokens, w.head_dim))
+        out.append(_to_bf16(x))
+    return out
+
+
 def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact upcast of a bf16 tensor to a float64 numpy array."""
     return t.to(torch.float32).numpy().astype(np.float64)

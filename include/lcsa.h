@@ -60,30 +60,47 @@ enum lcsa_status {
 #define LCSA_FLAG_PDL 2           /* launch as a programmatic dependent of the
                                      kernel that precedes the call in the stream,
                                      so that it starts while that kernel finishes.
-                                     lcsa_draft_mask / lcsa_attention wait for that
-                                     kernel (griddepcontrol.wait) before reading
-                                     the ring, the kept lists or the key means of
-                                     the newest q_layers layers, but read q_tok
-                                     (and the draft the key means of the layers
-                                     older than the newest max(q_layers,
-                                     cache->appended)) before the wait: set the
-                                     flag only when the preceding kernel writes
-                                     none of these (nor, for lcsa_attention,
-                                     out_tok or lse_opt), e.g. when it is the
-                                     cache append of the same chunk (before the
-                                     draft: it writes only the cache->appended
-                                     newest layers) or the draft (before the
-                                     attention).  lcsa_cache_append (flags
-                                     argument) writes the ring before the wait and
-                                     waits only at its end: set it only when the
-                                     preceding kernel writes neither k_tok nor v_tok
-                                     and the new layers fit the ring's spare slots
+                                     lcsa_draft_mask reads q_tok and writes
+                                     scores_opt / qmean_opt before waiting for
+                                     that kernel (griddepcontrol.wait), and reads
+                                     the key means and writes the kept lists only
+                                     after; lcsa_attention reads and writes
+                                     nothing before the wait.  Set the flag only
+                                     when the preceding kernel neither writes
+                                     q_tok nor touches scores_opt / qmean_opt,
+                                     e.g. when it is the cache append of the same
+                                     chunk (before the draft) or the draft
+                                     (before the attention).  lcsa_cache_append
+                                     (flags argument) writes the ring before the
+                                     wait and waits only at its end: set it only
+                                     when the preceding kernel writes neither
+                                     k_tok nor v_tok and the new layers fit the
+                                     ring's spare slots
                                      (n_layers <= capacity - window), e.g. when it
                                      is the previous chunk's lcsa_attention. */
 
 #define LCSA_HEAD_DIM 128
 #define LCSA_BLOCK_TOKENS 128
 #define LCSA_MAX_CANDIDATES 4096 /* allowed key blocks per query block */
+#define LCSA_MAX_SEGMENTS 256    /* segments of one lcsa_segment_mask call */
+
+/* Rotary position embedding of q and k (see lcsa_params.rope and the rope
+ * argument of lcsa_cache_append).  Named by the reading notes (背景, 关键设计
+ * 3) without a layout; the layout taken: each adjacent pair of dimensions
+ * (2i, 2i+1) of the 128-dim head turns by pos * w_i, the 64 pairs split into
+ * three axis bands: pairs [0, 22) over the latent frame's position in the
+ * stream (frame0 + the frame index inside the call's tensor), [22, 43) over the
+ * token row, [43, 64) over the token column; inside a band of n pairs
+ * w_i = base^(-i/n).  cos and sin are evaluated in fp64 and rounded to fp32,
+ * the rotation is computed in fp32 (each product and sum rounded once) and
+ * rounded to bf16: the rotated q and k are the bf16 values every later step
+ * (block means, scores, attention, the ring) uses. */
+typedef struct lcsa_rope {
+    float base;      /* e.g. 10000 (> 1); 0 disables the rotation */
+    int32_t frame0;  /* stream position of the first latent frame of the call's tokens, >= 0;
+                        every position (frame0 + frames of the call, token rows and
+                        columns) must stay <= 2^20, else LCSA_ERR_INVALID_ARG */
+} lcsa_rope;
 
 typedef struct lcsa_params {
     int32_t heads;       /* H >= 1 */
@@ -98,6 +115,8 @@ typedef struct lcsa_params {
                             row stride of kept_idx */
     float scale;         /* softmax scale; 0 -> 1/sqrt(head_dim) */
     int32_t flags;       /* LCSA_FLAG_*; 0 in normal use */
+    lcsa_rope rope;      /* rotation of q (draft and attention); base 0: none.
+                            frame0: stream position of q_tok's first frame */
 } lcsa_params;
 
 /* Ring of block-layers, caller-owned device buffers:
@@ -121,9 +140,6 @@ typedef struct lcsa_kv_cache {
     int32_t grid_h;
     int32_t grid_w;
     int32_t window;   /* 0 < window <= capacity, or 0 for capacity */
-    int32_t appended; /* layers written by the last lcsa_cache_append (set by
-                         it; start from 0): a draft chained after that append
-                         (LCSA_FLAG_PDL) reads them only after waiting for it */
 } lcsa_kv_cache;
 
 /*
@@ -137,13 +153,17 @@ typedef struct lcsa_kv_cache {
  *   flags: 0, LCSA_FLAG_PDL and/or LCSA_FLAG_FORCE_TIMEOUT (see there).
  *   d_status: device word (may be NULL); LCSA_ERR_TIMEOUT is OR-ed into it
  *   when a bounded wait for a copy gave up.
+ *   rope: NULL or base 0 for none; else k is rotated (lcsa_rope) before it is
+ *   stored and averaged, frame0 being the stream position of k_tok's first
+ *   frame.
  * The copies are TMA loads of whole blocks and bulk stores into the ring.
- * Updates cache->oldest/count/appended on the host when the copy is enqueued,
- * so calls on one cache must be serialised by the caller.
+ * Updates cache->oldest/count on the host when the copy is enqueued, so calls
+ * on one cache must be serialised by the caller.
  * 1 <= n_layers <= window.
  */
 int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok,
-                      int32_t n_layers, int32_t flags, int32_t *d_status, void *stream);
+                      int32_t n_layers, int32_t flags, const lcsa_rope *rope, int32_t *d_status,
+                      void *stream);
 
 /*
  * lcsa_draft_mask - the draft mask of learn.html 2.2, one row per
@@ -152,7 +172,8 @@ int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok
  * times 1/128); for every key block j allowed by the local window (same
  * spatial window on every layer, rule per local_mode) and by block causality
  * (key layer <= query layer): s = mean_q . kmean_j * scale, in fp32; keep the
- * min(topk, allowed) largest s, ties to the lower j.
+ * min(topk, allowed) largest s, ties to the lower j.  With p->rope, q is
+ * rotated (lcsa_rope) before its block means.
  *   q_tok      bf16 token layout [heads][2*q_layers][8*grid_h][8*grid_w][128]
  *   kept_idx   int32 [heads][q_layers*grid_h*grid_w][topk]: kept j ascending,
  *              padded with -1
@@ -178,6 +199,8 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
  *   out_tok  bf16, same layout as q_tok (written; may not alias q_tok)
  *   lse_opt  fp32 [heads][2*q_layers][8*grid_h][8*grid_w] or NULL: natural
  *            log of the softmax denominator of each query token
+ * With p->rope, the Q tiles are rotated (lcsa_rope) before the products (the
+ * keys were rotated by the cache append).
  * A row with kept_cnt == 0 gets zeros (lse -inf).  A kept index outside
  * [0, count*grid_h*grid_w) or a count outside [0, topk] sets
  * LCSA_ERR_BAD_INDEX and the row is written as if it kept nothing.
@@ -185,6 +208,30 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
 int lcsa_attention(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache *cache,
                    const int32_t *kept_idx, const int32_t *kept_cnt, void *out_tok,
                    float *lse_opt, int32_t *d_status, void *stream);
+
+/*
+ * lcsa_segment_mask - kept lists of the segment-masked dense attention of the
+ * reading notes' Stage-1 teacher (关键设计 1, the alpha_ij equation): over a
+ * packed sequence of segments (each one clip: a video, or an image as a
+ * single-frame video) every token attends to every token of its own segment
+ * and to no other.  The sequence is cut into 128-token tiles and segment s is
+ * the seg_tiles[s] tiles after those of segments 0 .. s-1 (so every segment
+ * holds a whole number of tiles, 128 * seg_tiles[s] tokens).  For every head
+ * h and query tile i of segment s it writes
+ *   kept_idx[h][i][0 .. n_s) = the segment's tiles in ascending order, then -1
+ *                             up to topk,   kept_cnt[h][i] = n_s = seg_tiles[s].
+ *   seg_tiles  HOST int32 [n_seg], each in [1, topk]; 1 <= n_seg <= LCSA_MAX_SEGMENTS
+ *   kept_idx   device int32 [heads][tiles][topk], kept_cnt device int32 [heads][tiles],
+ *              tiles = sum of seg_tiles; both 4-byte aligned
+ * lcsa_attention then computes the masked attention exactly: with q, k, v the
+ * packed sequence as bf16 [heads][128 * tiles][128] (the token layout with
+ * grid_h = grid_w = 1: a tile is one block-layer), k and v appended as
+ * `tiles` layers to a cache of grid 1 x 1, and params {grid 1 x 1,
+ * q_layers = tiles, topk}.  Asynchronous on `stream`; returns
+ * LCSA_ERR_INVALID_ARG (nothing enqueued) for a bad table or size.
+ */
+int lcsa_segment_mask(const int32_t *seg_tiles, int32_t n_seg, int32_t heads, int32_t topk, int32_t *kept_idx,
+                      int32_t *kept_cnt, void *stream);
 
 /* Human-readable name of a status code or of a device status word. */
 const char *lcsa_status_string(int code);

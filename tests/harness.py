@@ -69,27 +69,36 @@ class StepResult:
 
 
 def run_stream(w: W.Workload, n_steps: Optional[int] = None, n_rows: Optional[int] = None,
-               check_ring: bool = False, seed_rows: int = 0, on_step=None) -> List[StepResult]:
+               check_ring: bool = False, seed_rows: int = 0, on_step=None, rope_base: float = 0.0,
+               frame_offset: int = 0) -> List[StepResult]:
     """Run prefill + steps of ``w`` on the GPU and the oracle side by side.
 
     n_rows None compares the attention of every row.  With ``on_step`` each
-    step's result is handed to it and not kept (large workloads)."""
+    step's result is handed to it and not kept (large workloads).  With
+    ``rope_base`` q and k are rotated (the GPU in its kernels; the oracle
+    rotates them itself before its steps), the stream starting at frame
+    ``frame_offset``."""
     from diffusion_vsr_b200 import lcsa as L
 
     dev = torch.device("cuda")
     layer = L.LcsaLayer(w.heads, w.grid_h, w.grid_w, w.q_layers, w.kv_len, w.topk, w.local_range,
-                        w.local_mode, device=dev)
+                        w.local_mode, device=dev, rope_base=rope_base)
+    layer.frame = frame_offset
     ocache = O.KVCacheModel(w.capacity)
     prefill, steps = W.stream_plan(w)
     for p in prefill:
         _, k, v = W.gen_layers(w, p, 1, "kv")
+        frame0 = layer.frame
         layer.append(k.to(dev), v.to(dev))
-        ocache.append(f32(k), f32(v))
+        ocache.append(rotated(f32(k), frame0, rope_base), f32(v))
     results = []
     for p in steps[: (n_steps or len(steps))]:
         q, k, v = W.gen_layers(w, p, w.q_layers)
+        frame0 = layer.frame
+        layer.params.rope.frame0 = frame0
         res = step_both(w, layer.cache, ocache, layer.params, q, k, v, n_rows, check_ring,
-                        seed_rows + p, p, layer.status)
+                        seed_rows + p, p, layer.status, rope_base=rope_base, frame0=frame0)
+        layer.frame += k.shape[1]
         if on_step is not None:
             on_step(res)
             del res
@@ -99,7 +108,7 @@ def run_stream(w: W.Workload, n_steps: Optional[int] = None, n_rows: Optional[in
 
 
 def run_schedule(w: W.Workload, schedule: List[int], n_rows: Optional[int] = None,
-                 check_ring: bool = False) -> List[StepResult]:
+                 check_ring: bool = False, rope_base: float = 0.0) -> List[StepResult]:
     """A stream that starts from an empty cache of kv_len + 1 slots and appends
     ``schedule[i]`` block-layers at step i (e.g. a cold-start chunk of 3 layers,
     then chunks of 1), each step querying exactly the layers it appended."""
@@ -114,25 +123,34 @@ def run_schedule(w: W.Workload, schedule: List[int], n_rows: Optional[int] = Non
     results = []
     pos = 0
     for n_layers in schedule:
-        params = L.make_params(w.heads, w.grid_h, w.grid_w, n_layers, w.topk, w.local_range, w.local_mode)
+        params = L.make_params(w.heads, w.grid_h, w.grid_w, n_layers, w.topk, w.local_range, w.local_mode,
+                               rope_base=rope_base, rope_frame0=2 * pos)
         q, k, v = W.gen_layers(w, pos, n_layers)
-        results.append(step_both(w, cache, ocache, params, q, k, v, n_rows, check_ring, pos, pos, status))
+        results.append(step_both(w, cache, ocache, params, q, k, v, n_rows, check_ring, pos, pos, status,
+                                 rope_base=rope_base, frame0=2 * pos))
         pos += n_layers
     return results
 
 
+def rotated(x: np.ndarray, frame0: int, rope_base: float) -> np.ndarray:
+    """The oracle's RoPE of a token-layout tensor in the kernels' precision (or x unchanged)."""
+    return O.apply_rope(x, frame0, rope_base, "kernel") if rope_base else x
+
+
 def step_both(w: W.Workload, cache, ocache: O.KVCacheModel, params, q, k, v, n_rows, check_ring, seed,
-              position, status) -> StepResult:
+              position, status, rope_base: float = 0.0, frame0: int = 0) -> StepResult:
     """Append one chunk, then draft + attention on the GPU (own mask and the
-    oracle's mask) and the oracle step on the same inputs."""
+    oracle's mask) and the oracle step on the same inputs (rotated by the
+    oracle itself when ``rope_base`` is set)."""
     from diffusion_vsr_b200 import lcsa as L
 
     dev = torch.device("cuda")
     q_layers = q.shape[1] // 2
     Nq = q_layers * w.blocks_per_layer
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-    L.lcsa_cache_append(cache, kd, vd, d_status=status)
-    ocache.append(f32(k), f32(v))
+    L.lcsa_cache_append(cache, kd, vd, d_status=status,
+                        rope=L.lcsa_rope(rope_base, frame0) if rope_base else None)
+    ocache.append(rotated(f32(k), frame0, rope_base), f32(v))
     ring_ok = None
     kmean_err = None
     if check_ring:
@@ -148,8 +166,8 @@ def step_both(w: W.Workload, cache, ocache: O.KVCacheModel, params, q, k, v, n_r
     # oracle draft + selection on every row; attention on sampled rows
     rows = None if n_rows is None else sample_rows(w.heads, Nq, n_rows, seed)
     all_rows = [(h, i) for h in range(w.heads) for i in range(Nq)]
-    ref = O.lcsa_step(f32(q), ocache, w.grid_h, w.grid_w, w.topk, w.local_range, MODES[w.local_mode],
-                      rows=rows if rows is not None else all_rows)
+    ref = O.lcsa_step(rotated(f32(q), frame0, rope_base), ocache, w.grid_h, w.grid_w, w.topk, w.local_range,
+                      MODES[w.local_mode], rows=rows if rows is not None else all_rows)
     kept_o = torch.from_numpy(ref["kept_idx"]).to(dev)
     cnt_o = torch.from_numpy(ref["kept_cnt"]).to(dev)
     out_o = torch.empty_like(qd)

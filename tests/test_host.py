@@ -56,24 +56,13 @@ def _fake_cache(**kw):
 
 def test_cache_append_rejects_bad_arguments_without_touching_the_gpu(lib):
     c = _fake_cache()
-    assert lib.lcsa_cache_append(None, 0x40000, 0x50000, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
-    assert lib.lcsa_cache_append(ctypes.byref(c), None, 0x50000, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
-    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40008, 0x50000, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
-    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 5, 0, None, None) == L.LCSA_ERR_INVALID_ARG
-    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 0, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(None, 0x40000, 0x50000, 1, 0, None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), None, 0x50000, 1, 0, None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40008, 0x50000, 1, 0, None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 5, 0, None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 0, 0, None, None, None) == L.LCSA_ERR_INVALID_ARG
     bad = _fake_cache(count=5)
-    assert lib.lcsa_cache_append(ctypes.byref(bad), 0x40000, 0x50000, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
-
-
-def test_cache_appended_field_is_validated(lib):
-    # layers written by the last append: 0..capacity
-    z = ctypes.c_void_p(0x60000)
-    p = L.make_params(2, 4, 4, 1, 8)
-    for bad in (-1, 5):
-        c = _fake_cache(appended=bad)
-        assert lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None) == \
-            L.LCSA_ERR_INVALID_ARG
-        assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(bad), 0x40000, 0x50000, 1, 0, None, None, None) == L.LCSA_ERR_INVALID_ARG
 
 
 # A call that passes validation goes on to launch a kernel: with the fake
@@ -86,9 +75,9 @@ no_gpu_only = pytest.mark.skipif(torch.cuda.is_available(),
 def test_append_of_more_than_sixteen_layers_passes_validation(lib):
     # the ring slots are computed on the device: any n_layers <= window is accepted
     c = _fake_cache(capacity=40, window=40, count=0, heads=1)
-    rc = lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 33, 0, None, None)
+    rc = lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 33, 0, None, None, None)
     assert rc != L.LCSA_ERR_INVALID_ARG
-    assert c.count == 0 and c.appended == 0  # nothing enqueued without a GPU: state unchanged
+    assert c.count == 0  # nothing enqueued without a GPU: state unchanged
 
 
 @no_gpu_only
@@ -96,15 +85,15 @@ def test_cache_window_and_overlap_rules(lib):
     k, v = 0x40000, 0x50000
     # at most `window` layers resident, window <= capacity
     wide = _fake_cache(capacity=5, window=6, count=4)
-    assert lib.lcsa_cache_append(ctypes.byref(wide), k, v, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(wide), k, v, 1, 0, None, None, None) == L.LCSA_ERR_INVALID_ARG
     over = _fake_cache(capacity=5, window=4, count=5)
-    assert lib.lcsa_cache_append(ctypes.byref(over), k, v, 1, 0, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(over), k, v, 1, 0, None, None, None) == L.LCSA_ERR_INVALID_ARG
     # an append overlapping the previous step must fit the spare slots (5 - 4 = 1 here)
     ok = _fake_cache(capacity=5, window=4, count=4)
-    assert lib.lcsa_cache_append(ctypes.byref(ok), k, v, 2, L.LCSA_FLAG_PDL, None, None) == L.LCSA_ERR_INVALID_ARG
-    assert lib.lcsa_cache_append(ctypes.byref(ok), k, v, 1, L.LCSA_FLAG_PDL, None, None) != L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(ok), k, v, 2, L.LCSA_FLAG_PDL, None, None, None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_cache_append(ctypes.byref(ok), k, v, 1, L.LCSA_FLAG_PDL, None, None, None) != L.LCSA_ERR_INVALID_ARG
     no_spare = _fake_cache(capacity=4, window=0, count=4)
-    assert lib.lcsa_cache_append(ctypes.byref(no_spare), k, v, 1, L.LCSA_FLAG_PDL, None, None) == \
+    assert lib.lcsa_cache_append(ctypes.byref(no_spare), k, v, 1, L.LCSA_FLAG_PDL, None, None, None) == \
         L.LCSA_ERR_INVALID_ARG
 
 
@@ -119,6 +108,22 @@ def test_draft_and_attention_reject_bad_params(lib, field, value):
         L.LCSA_ERR_INVALID_ARG
     assert lib.lcsa_attention(ctypes.byref(p), z, ctypes.byref(c), z, z, ctypes.c_void_p(0x70000), None, None,
                               None) == L.LCSA_ERR_INVALID_ARG
+
+
+@no_gpu_only
+def test_rope_arguments_are_validated(lib):
+    z = ctypes.c_void_p(0x60000)
+    c = _fake_cache()
+    for base, frame0, ok in [(10000.0, 0, True), (0.0, -5, True), (1.0, 0, False), (-3.0, 0, False),
+                             (float("inf"), 0, False), (10000.0, -1, False), (10000.0, (1 << 20) - 2, True),
+                             (10000.0, (1 << 20) - 1, False)]:
+        p = L.make_params(2, 4, 4, 1, 8, rope_base=base, rope_frame0=frame0)
+        rc = lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None)
+        assert (rc != L.LCSA_ERR_INVALID_ARG) == ok, (base, frame0, rc)
+        r = L.lcsa_rope(base, frame0)
+        rc = lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 1, 0, ctypes.byref(r), None, None)
+        if not ok:
+            assert rc == L.LCSA_ERR_INVALID_ARG, (base, frame0)
 
 
 def test_draft_rejects_too_many_candidates(lib):
@@ -136,6 +141,24 @@ def test_attention_rejects_aliased_output(lib):
     z = ctypes.c_void_p(0x60000)
     assert lib.lcsa_attention(ctypes.byref(p), z, ctypes.byref(c), z, z, z, None, None, None) == \
         L.LCSA_ERR_INVALID_ARG
+
+
+def test_segment_mask_rejects_bad_tables(lib):
+    z = ctypes.c_void_p(0x60000)
+
+    def call(tiles, heads=2, topk=8, kept=z, cnt=z):
+        arr = (ctypes.c_int32 * max(len(tiles), 1))(*tiles)
+        return lib.lcsa_segment_mask(arr if tiles is not None else None, len(tiles), heads, topk, kept, cnt, None)
+
+    assert call([]) == L.LCSA_ERR_INVALID_ARG                    # no segment
+    assert call([3, 0, 2]) == L.LCSA_ERR_INVALID_ARG             # empty segment
+    assert call([3, 9]) == L.LCSA_ERR_INVALID_ARG                # longer than topk
+    assert call([3, 2], heads=0) == L.LCSA_ERR_INVALID_ARG
+    assert call([3, 2], topk=0) == L.LCSA_ERR_INVALID_ARG
+    assert call([1] * (L.LCSA_MAX_SEGMENTS + 1)) == L.LCSA_ERR_INVALID_ARG
+    assert call([3, 2], kept=ctypes.c_void_p(0x60002)) == L.LCSA_ERR_INVALID_ARG  # misaligned
+    assert call([3, 2], cnt=None) == L.LCSA_ERR_INVALID_ARG
+    assert lib.lcsa_segment_mask(None, 2, 2, 8, z, z, None) == L.LCSA_ERR_INVALID_ARG
 
 
 def test_binding_refuses_cpu_tensors():
