@@ -99,43 +99,27 @@ cudaError_t launch_attention(const CUtensorMap &tm_q, const CUtensorMap &tm_k, c
                              const CUtensorMap &tm_o, const AttnArgs &a, const AttnRope &rope, bool pdl, void *out,
                              const DeviceInfo &dev, cudaStream_t stream);
 
-// Draft mask: q block means, scores over allowed candidates, top-k.  One CTA
-// per tile of tile_h x tile_w query blocks of one (head, query layer); rmax
-// (>= tile rows, one of 4, 8, 12, 16) and kpt (union keys per thread and
-// round, 1..3) select the kernel instance.
+// Draft mask: q block means, scores over allowed candidates, top-k.
 struct DraftArgs {
+    const uint16_t *q;     // bf16 token layout
     const float *kmean;    // [cap][H][nblk][128]
-    int32_t heads, grid_h, grid_w, nblk, q_layers;
+    int32_t heads, grid_h, grid_w, nblk, q_layers, tq, tok_h, tok_w;
     int32_t capacity, oldest, count;
+    int32_t fresh_layers;  // newest layers the preceding kernel may still be writing (PDL)
     int32_t local_range, local_mode, topk;
     int32_t cand_cap;      // most allowed candidates of a row, rounded up to 32
-    int32_t tile_h, tile_w, tiles_y, tiles_x;
-    int32_t rmax, kpt;
-    // ceil(2^32 / d) for d = tiles_y * tiles_x, q_layers, tiles_x: n / d = (n * m) >> 32
-    uint64_t m_tiles, m_ql, m_tiles_x;
+    uint64_t m_nq, m_nblk, m_gw;  // multiply-high multipliers of q_layers*nblk, nblk, grid_w
     float scale;
     int32_t *kept_idx;
     int32_t *kept_cnt;
     float *scores;         // may be null
     float *qmean;          // may be null
-    int32_t *status;       // may be null
-    uint64_t timeout_ns;
+    int32_t *status;
     float rope_base;       // 0: no rotation of q
     int32_t rope_frame0;   // stream position of q's first frame
-    int32_t rope_entries;  // rotation table entries of a tile (0 without rotation)
 };
 
-// Entries of a draft CTA's rotation table for tiles of tile_h x tile_w blocks.
-inline int draft_rope_entries(int tile_h, int tile_w) { return 2 * 22 + 8 * (tile_h + tile_w) * 21; }
-
-// Shared memory of the draft kernel instance (rmax, kpt) for rows of at most
-// cand_cap candidates, alignment slack included (0 for an unknown instance).
-size_t draft_smem_bytes(int rmax, int kpt, int cand_cap, int rope_entries);
-
-// tm_q: rank-4 map over q in token layout with a whole-block box (128 dims,
-// 8, 8, 2 frames), no swizzle.
-cudaError_t launch_draft(const CUtensorMap &tm_q, const DraftArgs &a, bool pdl, const DeviceInfo &dev,
-                         cudaStream_t stream);
+cudaError_t launch_draft(const DraftArgs &a, bool pdl, const DeviceInfo &dev, cudaStream_t stream);
 
 // Cache append: token layout -> block layout ring slots + k block means.
 struct AppendArgs {

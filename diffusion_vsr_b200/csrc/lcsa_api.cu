@@ -86,6 +86,7 @@ int check_cache(const lcsa_kv_cache *c) {
     if (c->window < 0 || c->window > c->capacity) return LCSA_ERR_INVALID_ARG;
     if (c->count < 0 || c->count > window_of(c) || c->oldest < 0 || c->oldest >= c->capacity)
         return LCSA_ERR_INVALID_ARG;
+    if (c->appended < 0 || c->appended > c->capacity) return LCSA_ERR_INVALID_ARG;
     // every token row index of the ring must fit a signed 32-bit TMA coordinate
     const int64_t rows = static_cast<int64_t>(c->capacity) * c->heads * c->grid_h * c->grid_w * kBlockTokens;
     if (rows >= (int64_t(1) << 31)) return LCSA_ERR_INVALID_ARG;
@@ -232,77 +233,6 @@ bool make_ring_map(CUtensorMap *m, const void *base, int64_t rows) {
                       [&](CUtensorMap *o) { return encode_ring_map(o, base, rows); });
 }
 
-// Allowed block range [lo, hi) along one axis (the draft kernel's window rule).
-void window_1d_host(int i, int n, int r, int mode, int &lo, int &hi) {
-    if (r <= 0 || (mode == 0 && n <= r)) {
-        lo = 0;
-        hi = n;
-        return;
-    }
-    const int h = r / 2;
-    if (mode == 0) {
-        lo = std::min(std::max(i - h, 0), n - r);
-        hi = lo + r;
-    } else {
-        lo = std::max(i - h, 0);
-        hi = std::min(i + h + 1, n);
-    }
-}
-
-// Widest union of the windows of `t` consecutive blocks along an axis of n.
-int union_span(int n, int t, int r, int mode) {
-    int best = 0;
-    for (int i0 = 0; i0 < n; i0 += t) {
-        int lo, hi, lo2, hi2;
-        window_1d_host(i0, n, r, mode, lo, hi);
-        window_1d_host(std::min(i0 + t, n) - 1, n, r, mode, lo2, hi2);
-        best = std::max(best, hi2 - lo);
-    }
-    return best;
-}
-
-struct DraftTiling {
-    int th, tw, rmax, kpt;
-};
-
-// Tile of query blocks per draft CTA.  Estimated SM cycles per CTA: its q
-// blocks from DRAM (~1,450 cycles per 32 KB block at an even share of the HBM
-// bandwidth), the staged union keys (~7 cycles each from L2) and their products
-// with every block of the tile (~2 cycles per block and key), the selection
-// (~300 cycles per block); CTAs run two per SM when their shared memory allows.
-// The tile with the fewest estimated cycles over all waves wins.
-DraftTiling choose_draft_tiling(const lcsa_params *p, const lcsa_kv_cache *c, int cand_cap, int sms) {
-    DraftTiling best{1, 1, 4, 1};
-    double best_cost = 1e300;
-    const int max_smem = 227 * 1024;
-    for (int th = 1; th <= std::min(p->grid_h, 16); ++th) {
-        for (int tw = 1; tw <= std::min(p->grid_w, 16); ++tw) {
-            const int R = th * tw;
-            if (R > 16) continue;
-            const int rmax = R <= 4 ? 4 : R <= 8 ? 8 : R <= 12 ? 12 : 16;
-            const int64_t utotal = static_cast<int64_t>(c->count) * union_span(p->grid_h, th, p->local_range, p->local_mode) *
-                                   union_span(p->grid_w, tw, p->local_range, p->local_mode);
-            const int kpt = static_cast<int>(std::min<int64_t>(3, std::max<int64_t>(1, (utotal + 255) / 256)));
-            const size_t smem = lcsa::draft_smem_bytes(rmax, kpt, cand_cap,
-                                                       p->rope.base != 0.f ? lcsa::draft_rope_entries(th, tw) : 0);
-            if (smem == 0 || smem > static_cast<size_t>(max_smem)) continue;
-            const int64_t rounds = (utotal + 256 * kpt - 1) / (256 * kpt);
-            const int64_t ctas = static_cast<int64_t>(p->heads) * p->q_layers * ((p->grid_h + th - 1) / th) *
-                                 ((p->grid_w + tw - 1) / tw);
-            const int per_sm = smem <= 113 * 1024 ? 2 : 1;
-            const int64_t waves = (ctas + static_cast<int64_t>(sms) * per_sm - 1) / (static_cast<int64_t>(sms) * per_sm);
-            const double compute = static_cast<double>(rounds) * 256 * kpt * (2.0 * R + 7.0) + 300.0 * R;
-            const double dram = 1450.0 * R;
-            const double cost = static_cast<double>(waves) * std::max(compute, dram) * (per_sm == 2 ? 1.0 : 1.3);
-            if (cost < best_cost) {
-                best_cost = cost;
-                best = DraftTiling{th, tw, rmax, kpt};
-            }
-        }
-    }
-    return best;
-}
-
 }  // namespace
 
 extern "C" {
@@ -376,6 +306,7 @@ int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok
         return LCSA_ERR_CUDA;
     cache->oldest = oldest;
     cache->count = count;
+    cache->appended = n_layers;
     return LCSA_OK;
 }
 
@@ -390,44 +321,35 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
     const lcsa::DeviceInfo *dev = nullptr;
     if ((rc = device_of(&dev)) != LCSA_OK) return rc;
 
-    const int nblk = p->grid_h * p->grid_w;
-    const int cand_cap = static_cast<int>((cand + 31) / 32 * 32);
-    // union keys per CTA and every index the kernel divides must stay below 2^16
-    if (static_cast<int64_t>(cache->count) * nblk >= (1 << 16)) return LCSA_ERR_INVALID_ARG;
-    const DraftTiling tl = choose_draft_tiling(p, cache, cand_cap, dev->sms);
-    const int64_t frames = static_cast<int64_t>(p->heads) * 2 * p->q_layers;
-    CUtensorMap tq;
-    if (!make_chunk_map(&tq, q_tok, frames, 8 * p->grid_h, 8 * p->grid_w)) return LCSA_ERR_CUDA;
-
     lcsa::DraftArgs a{};
+    a.q = static_cast<const uint16_t *>(q_tok);
     a.kmean = cache->kmean;
     a.heads = p->heads;
     a.grid_h = p->grid_h;
     a.grid_w = p->grid_w;
-    a.nblk = nblk;
+    a.nblk = p->grid_h * p->grid_w;
     a.q_layers = p->q_layers;
+    a.tq = 2 * p->q_layers;
+    a.tok_h = 8 * p->grid_h;
+    a.tok_w = 8 * p->grid_w;
     a.capacity = cache->capacity;
     a.oldest = cache->oldest;
     a.count = cache->count;
+    // chained after an append (LCSA_FLAG_PDL), the layers it wrote are read only
+    // after waiting for it: the query layers, and every layer of that append
+    a.fresh_layers = std::max(p->q_layers, cache->appended);
     a.local_range = p->local_range;
     a.local_mode = p->local_mode;
     a.topk = p->topk;
-    a.cand_cap = cand_cap;
-    a.tile_h = tl.th;
-    a.tile_w = tl.tw;
-    a.tiles_y = (p->grid_h + tl.th - 1) / tl.th;
-    a.tiles_x = (p->grid_w + tl.tw - 1) / tl.tw;
-    a.rmax = tl.rmax;
-    a.kpt = tl.kpt;
+    a.cand_cap = static_cast<int32_t>((cand + 31) / 32 * 32);
     {
-        // CTA decomposition by multiply-high division, exact while dividend x divisor <= 2^32
-        const int64_t per = static_cast<int64_t>(a.tiles_y) * a.tiles_x;
-        const int64_t grid = static_cast<int64_t>(p->heads) * p->q_layers * per;
-        if (grid * per > (1ll << 32) || grid * p->q_layers > (1ll << 32) || per * a.tiles_x > (1ll << 32))
+        // row decomposition by multiply-high division, exact while dividend x divisor <= 2^32
+        const int64_t nq = static_cast<int64_t>(p->q_layers) * a.nblk;
+        if (static_cast<int64_t>(p->heads) * nq * nq > (1ll << 32) || nq * a.nblk > (1ll << 32))
             return LCSA_ERR_INVALID_ARG;
-        a.m_tiles = lcsa::div_magic_host(static_cast<uint32_t>(per));
-        a.m_ql = lcsa::div_magic_host(static_cast<uint32_t>(p->q_layers));
-        a.m_tiles_x = lcsa::div_magic_host(static_cast<uint32_t>(a.tiles_x));
+        a.m_nq = lcsa::div_magic_host(static_cast<uint32_t>(nq));
+        a.m_nblk = lcsa::div_magic_host(static_cast<uint32_t>(a.nblk));
+        a.m_gw = lcsa::div_magic_host(static_cast<uint32_t>(a.grid_w));
     }
     a.scale = eff_scale(p);
     a.kept_idx = kept_idx;
@@ -435,12 +357,9 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
     a.scores = scores_opt;
     a.qmean = qmean_opt;
     a.status = d_status;
-    a.timeout_ns = lcsa::kWatchdogNs;
     a.rope_base = p->rope.base;
     a.rope_frame0 = p->rope.frame0;
-    a.rope_entries = p->rope.base != 0.f ? lcsa::draft_rope_entries(tl.th, tl.tw) : 0;
-    if (lcsa::launch_draft(tq, a, (p->flags & LCSA_FLAG_PDL) != 0, *dev, static_cast<cudaStream_t>(stream)) !=
-        cudaSuccess)
+    if (lcsa::launch_draft(a, (p->flags & LCSA_FLAG_PDL) != 0, *dev, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LCSA_ERR_CUDA;
     return LCSA_OK;
 }

@@ -47,7 +47,7 @@ class lcsa_kv_cache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("kmean", ctypes.c_void_p),
                 ("capacity", ctypes.c_int32), ("oldest", ctypes.c_int32), ("count", ctypes.c_int32),
                 ("heads", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
-                ("window", ctypes.c_int32)]
+                ("window", ctypes.c_int32), ("appended", ctypes.c_int32)]
 
 
 class LcsaError(RuntimeError):
@@ -154,6 +154,7 @@ class KVCache:
     def reset(self) -> None:
         self.desc.oldest = 0
         self.desc.count = 0
+        self.desc.appended = 0
 
 
 def lcsa_cache_append(cache: KVCache, k_tok: torch.Tensor, v_tok: torch.Tensor, n_layers: Optional[int] = None,

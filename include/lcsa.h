@@ -60,17 +60,22 @@ enum lcsa_status {
 #define LCSA_FLAG_PDL 2           /* launch as a programmatic dependent of the
                                      kernel that precedes the call in the stream,
                                      so that it starts while that kernel finishes.
-                                     lcsa_draft_mask reads q_tok and writes
-                                     scores_opt / qmean_opt before waiting for
-                                     that kernel (griddepcontrol.wait), and reads
-                                     the key means and writes the kept lists only
+                                     lcsa_draft_mask reads q_tok, writes
+                                     scores_opt / qmean_opt and reads the key
+                                     means of the layers older than the newest
+                                     max(q_layers, cache->appended) before
+                                     waiting for that kernel
+                                     (griddepcontrol.wait), and reads the other
+                                     key means and writes the kept lists only
                                      after; lcsa_attention reads and writes
                                      nothing before the wait.  Set the flag only
                                      when the preceding kernel neither writes
-                                     q_tok nor touches scores_opt / qmean_opt,
-                                     e.g. when it is the cache append of the same
-                                     chunk (before the draft) or the draft
-                                     (before the attention).  lcsa_cache_append
+                                     q_tok or those older key means nor touches
+                                     scores_opt / qmean_opt, e.g. when it is the
+                                     cache append of the same chunk (before the
+                                     draft: it writes only the cache->appended
+                                     newest layers) or the draft (before the
+                                     attention).  lcsa_cache_append
                                      (flags argument) writes the ring before the
                                      wait and waits only at its end: set it only
                                      when the preceding kernel writes neither
@@ -140,6 +145,9 @@ typedef struct lcsa_kv_cache {
     int32_t grid_h;
     int32_t grid_w;
     int32_t window;   /* 0 < window <= capacity, or 0 for capacity */
+    int32_t appended; /* layers written by the last lcsa_cache_append (set by
+                         it; start from 0): a draft chained after that append
+                         (LCSA_FLAG_PDL) reads them only after waiting for it */
 } lcsa_kv_cache;
 
 /*
@@ -157,8 +165,8 @@ typedef struct lcsa_kv_cache {
  *   stored and averaged, frame0 being the stream position of k_tok's first
  *   frame.
  * The copies are TMA loads of whole blocks and bulk stores into the ring.
- * Updates cache->oldest/count on the host when the copy is enqueued, so calls
- * on one cache must be serialised by the caller.
+ * Updates cache->oldest/count/appended on the host when the copy is enqueued,
+ * so calls on one cache must be serialised by the caller.
  * 1 <= n_layers <= window.
  */
 int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok,

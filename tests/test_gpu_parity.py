@@ -214,8 +214,9 @@ def test_programmatic_dependent_launch_matches_plain_launches():
 def test_chained_draft_after_multi_layer_append_matches_plain_launches():
     # A cold-start append of 3 block-layers, then a draft of only the newest
     # layer launched as a programmatic dependent of that append: the draft must
-    # not read the key means of any of the 3 layers before the append completed.
-    # Kept lists and scores equal those of plain launches bit for bit.
+    # not read the key means of any of the 3 layers before the append completed
+    # (the cache records how many layers the append wrote).  Kept lists and
+    # scores equal those of plain launches bit for bit.
     import dataclasses
     L = _lib()
     w = W.WORKLOADS["768x1280"]
@@ -234,7 +235,7 @@ def test_chained_draft_after_multi_layer_append_matches_plain_launches():
         for _ in range(3):  # the same append and draft, repeated
             cache.reset()
             L.lcsa_cache_append(cache, k3, v3, d_status=st)
-            assert cache.count == 3
+            assert cache.desc.appended == 3 and cache.count == 3
             L.lcsa_draft_mask(p, q_new, cache, kept, cnt, scores, d_status=st)
         torch.cuda.synchronize()
         assert st.item() == 0

@@ -65,6 +65,18 @@ def test_cache_append_rejects_bad_arguments_without_touching_the_gpu(lib):
     assert lib.lcsa_cache_append(ctypes.byref(bad), 0x40000, 0x50000, 1, 0, None, None, None) == L.LCSA_ERR_INVALID_ARG
 
 
+def test_cache_appended_field_is_validated(lib):
+    # layers written by the last append: 0..capacity
+    z = ctypes.c_void_p(0x60000)
+    p = L.make_params(2, 4, 4, 1, 8)
+    for bad in (-1, 5):
+        c = _fake_cache(appended=bad)
+        assert lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None) == \
+            L.LCSA_ERR_INVALID_ARG
+        assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 1, 0, None, None, None) == \
+            L.LCSA_ERR_INVALID_ARG
+
+
 # A call that passes validation goes on to launch a kernel: with the fake
 # pointers of these tests that must only happen where no GPU exists.
 no_gpu_only = pytest.mark.skipif(torch.cuda.is_available(),
