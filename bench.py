@@ -10,7 +10,10 @@ blocks), local range 11, topk 20.
 
 Prints one JSON line.  ``value`` is the effective throughput in TFLOP/s
 counted over kept tiles only (4 * 128^3 flops per tile); ``ms_per_step`` is
-ms per chunk.  ``--sweep`` prints one such line per workload instead.
+ms per chunk.  ``--sweep`` prints one such line per workload instead, plus one line for the
+segment-masked dense attention of the Stage-1 teacher (``--segments``: a
+packed sequence of images and videos, each attending only to itself).
+``--rope BASE`` runs the streaming step with RoPE applied to q and k.
 ``--impl reference`` times the fp64 CPU oracle (rank 0 only): each step is
 one whole chunk of a slice of the heads (append, draft and attention of every
 row of those heads), sized so that the run ends within a few minutes.
@@ -49,6 +52,8 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 SWEEP = (("768x1280", 0), ("768x1408", 0), ("1536x2688", 0), ("4k", 8), ("4k", 16), ("4k", 32))
+SWEEP_SEGMENTS = "768x1280"
+SEGMENT_METRIC = "segment-masked dense attention (Stage-1 teacher): effective TFLOP/s over the segments' tiles"
 REFERENCE_BUDGET_S = 150.0  # wall-clock budget of a whole reference-arm run (warm-up + timed steps)
 E2E_MIN_STEPS = 50
 
@@ -65,6 +70,9 @@ def parse_args(argv=None):
                     help="distinct chunk buffers rotated across steps (fewer: a reduced case for ncu captures)")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per workload (768x1280, 768x1408, 1536x2688, 4K topk 8/16/32)")
+    ap.add_argument("--rope", type=float, default=0.0, help="RoPE base for q and k (0: no rotation)")
+    ap.add_argument("--segments", default=None, choices=sorted(W.SEGMENT_WORKLOADS),
+                    help="time the segment-masked dense attention of this packed sequence of clips instead")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
@@ -178,9 +186,10 @@ def aggregate_tflops(world: int, flops_per_rank_step: float, ms_per_step: float)
     return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
 
 
-def bench_config(w: W.Workload, kept_tiles: int, world: int) -> dict:
+def bench_config(w: W.Workload, kept_tiles: int, world: int, rope: float = 0.0) -> dict:
     """The workload a line is measured on; both arms print this same dict."""
-    return {
+    extra = {"rope_base": rope} if rope else {}
+    return {**extra,
         "workload": f"{w.name} streaming chunk, one DiT attention layer",
         "heads": w.heads, "head_dim": w.head_dim, "query_blocks": w.n_query_blocks, "key_blocks": w.n_key_blocks,
         "kv_len_layers": w.kv_len, "local_range": w.local_range,
@@ -244,7 +253,7 @@ def measure_lcsa(w: W.Workload, args, world: int, local_rank: int, dev, with_e2e
     host = [W.gen_layers(w, p, w.q_layers) for p in positions]
     chunks = [[t.to(dev) for t in c] for c in host]
     layer = L.LcsaLayer(w.heads, w.grid_h, w.grid_w, w.q_layers, w.kv_len, w.topk, w.local_range, w.local_mode,
-                        device=dev)
+                        device=dev, rope_base=args.rope)
     for p in prefill:
         _, k, v = W.gen_layers(w, p, 1, "kv")
         layer.append(k.to(dev), v.to(dev))
@@ -262,12 +271,25 @@ def measure_lcsa(w: W.Workload, args, world: int, local_rank: int, dev, with_e2e
         # the same three calls without programmatic dependence, with events between
         # them: per-kernel times for the roofline
         q, k, v = chunks[i % n_bufs]
+        frame0 = layer.frame
+        layer.params.rope.frame0 = frame0
         ev[0].record(stream)
-        L.lcsa_cache_append(layer.cache, k, v, d_status=layer.status)
+        L.lcsa_cache_append(layer.cache, k, v, d_status=layer.status, rope=layer._rope(frame0))
+        layer.frame += k.shape[1]
         ev[1].record(stream)
-        L.lcsa_draft_mask(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, d_status=layer.status)
+        if args.rope:
+            # as LcsaLayer.step: the draft stores the rotated q, the attention reads it
+            if layer.q_rot is None:
+                layer.q_rot = torch.empty_like(q)
+            L.lcsa_draft_mask(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, d_status=layer.status,
+                              q_rot=layer.q_rot)
+            attn_params, attn_q = L.make_params(w.heads, w.grid_h, w.grid_w, w.q_layers, w.topk, w.local_range,
+                                                w.local_mode), layer.q_rot
+        else:
+            L.lcsa_draft_mask(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, d_status=layer.status)
+            attn_params, attn_q = layer.params, q
         ev[2].record(stream)
-        L.lcsa_attention(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, out, d_status=layer.status)
+        L.lcsa_attention(attn_params, attn_q, layer.cache, layer.kept_idx, layer.kept_cnt, out, d_status=layer.status)
         ev[3].record(stream)
 
     for i in range(args.warmup):
@@ -337,7 +359,7 @@ def measure_lcsa(w: W.Workload, args, world: int, local_rank: int, dev, with_e2e
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 q/k/v" + (" with per-head low-rank block bias" if w.lowrank else "")
                 + "; random, no weights)",
-        "config": bench_config(w, kept_tiles, world),
+        "config": bench_config(w, kept_tiles, world, args.rope),
         "inputs": f"{n_bufs} distinct chunk buffers rotated, ring "
                   f"{(layer.cache.k.numel() + layer.cache.v.numel()) * 2 / 1e6:.0f} MB "
                   f"({layer.cache.desc.capacity} slots, {w.capacity} resident)",
@@ -421,13 +443,112 @@ def run_e2e(args, L, layer, host, dev, stream, step_flops, world):
             "overlap": "H2D of chunk i+1 and D2H of chunk i-1 overlap chunk i's kernels (two copy streams)"}
 
 
+def measure_segments(sw: W.SegmentWorkload, args, world: int, local_rank: int, dev):
+    """The Stage-1 teacher's segment-masked dense attention of a packed sequence
+    of clips: a step appends the pack's k/v (one ring layer per 128-token tile)
+    and runs the attention over the segment kept lists (every tile of the own
+    segment), both through the C ABI; the kept lists are built once."""
+    from diffusion_vsr_b200 import lcsa as L
+
+    seg = L.SegmentAttention(sw.heads, sw.seg_tiles, device=dev)
+    q, k, v = [t.to(dev) for t in W.gen_segments(sw)]
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        seg.run(q, k, v, out)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(args.steps):
+            seg.run(q, k, v, out)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_step = max_over_ranks(t0.elapsed_time(t1), dev) / args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for e in evs:
+        seg.cache.reset()
+        e[0].record(stream)
+        L.lcsa_cache_append(seg.cache, k, v, n_layers=seg.tiles, d_status=seg.status)
+        e[1].record(stream)
+        L.lcsa_attention(seg.params, q, seg.cache, seg.kept_idx, seg.kept_cnt, out, d_status=seg.status)
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    status = int(seg.status.item())
+    if status != 0:
+        raise RuntimeError(f"device status {L.status_string(status)}")
+    t_append = [e[0].elapsed_time(e[1]) for e in evs]
+    t_attn = [e[1].elapsed_time(e[2]) for e in evs]
+    pk = peaks()
+    flops = sw.kept_tiles * W.flops_per_tile()
+    tensor_bytes = sw.heads * sw.tokens * 128 * 2  # one of q, k, v, out
+    attn_ms = statistics.mean(t_attn)
+    append_ms = statistics.mean(t_append)
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    # the attention reads q and the whole ring (every key tile is some row's kept tile) and writes out
+    attn_bytes = 4 * tensor_bytes + sw.heads * seg.tiles * (seg.topk + 1) * 4
+    attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9
+    append_bytes = 4 * tensor_bytes + sw.heads * seg.tiles * 128 * 4
+    tensor_frac = attn_tflops / pk["bf16_tflops"]
+    hbm_frac = attn_gbs / pk["hbm_gbs"]
+    return {
+        "metric": SEGMENT_METRIC,
+        "value": round(aggregate_tflops(world, flops, ms_step), 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v; random, no weights)",
+        "config": {
+            "workload": f"segments {sw.name}: packed clips (latent frames, token rows, token columns) "
+                        f"{[list(c) for c in sw.clips]}",
+            "heads": sw.heads, "head_dim": sw.head_dim, "tokens": sw.tokens, "segment_tiles": sw.seg_tiles,
+            "kept_tiles": sw.kept_tiles, "tflop_per_step": round(flops / 1e12, 5),
+            "l2": "inputs larger than L2 (126 MB): q, k, v, out and the ring each "
+                  f"{tensor_bytes / 1e6:.0f} MB",
+            "parallelism": f"replicas x{world}" if world > 1 else "single replica",
+        },
+        "launch": "per step: lcsa_cache_append of the whole pack (one ring layer per tile), then lcsa_attention "
+                  "over the segment kept lists (built once by lcsa_segment_mask); per-kernel times from a "
+                  "separate pass with events between the calls",
+        "roofline": {
+            "kernel": "lcsa_attention (tcgen05 block-sparse attention)", "bound": "tensor",
+            "achieved": round(attn_tflops, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(tensor_frac, 4), "peak_source": f"{pk['source']} dense bf16 (burst)", "traffic": None,
+            "algorithmic_flops_per_launch": flops, "avg_launch_ms": round(attn_ms, 5),
+            "hbm_bound": {"achieved": round(attn_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                          "frac": round(hbm_frac, 4), "algorithmic_bytes_per_launch": attn_bytes,
+                          "bytes": "Q + O + the K/V ring + kept lists"},
+            "binding": "tensor" if tensor_frac >= hbm_frac else "hbm",
+        },
+        "kernels": {
+            "attention_ms": round(attn_ms, 5), "attention_median_ms": round(statistics.median(t_attn), 5),
+            "cache_append_ms": round(append_ms, 5),
+            "cache_append_median_ms": round(statistics.median(t_append), 5),
+            "cache_append_gbs": round(append_bytes / (append_ms * 1e-3) / 1e9, 1),
+            "cache_append_bytes": append_bytes,
+        },
+        "clocks": clocks.summary(),
+        "gpu_launches": 2 * args.steps,
+    }
+
+
 def run_lcsa(args, rank: int, world: int, local_rank: int):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    if args.segments:
+        return [measure_segments(W.SEGMENT_WORKLOADS[args.segments], args, world, local_rank, dev)]
     if args.sweep:
         out = []
         for name, topk in SWEEP:
             out.append(measure_lcsa(workload_of(name, topk), args, world, local_rank, dev, with_e2e=False))
+        out.append(measure_segments(W.SEGMENT_WORKLOADS[SWEEP_SEGMENTS], args, world, local_rank, dev))
         return out
     return [measure_lcsa(workload(args), args, world, local_rank, dev, with_e2e=not args.no_e2e)]
 
@@ -577,7 +698,7 @@ def main(argv=None):
     try:
         results = run_lcsa(args, rank, world, local_rank)
         if rank == 0:
-            if not args.no_cpu_baseline and not args.sweep:
+            if not args.no_cpu_baseline and not args.sweep and not args.segments:
                 results[0]["cpu_baseline"] = cpu_baseline(workload(args))
             for r in results:
                 print(json.dumps(r), flush=True)

@@ -16,7 +16,8 @@
 //     the 8 partial sums are added in a fixed tree order, times 1/128
 //     (deterministic); with RoPE every pair of q is rotated (and rounded to
 //     bf16) before it is summed, from a table of the block's (cos, sin) that
-//     the CTA builds while its loads are in flight;
+//     the CTA builds while its loads are in flight, and the rotated q is
+//     stored for the attention when the caller asks for it;
 //  2. the allowed candidates, enumerated in ascending key index (layer, then
 //     window row, then window column), eight per warp at a time: each 512-byte
 //     key mean is one coalesced warp load, dotted with the q mean in fp32
@@ -105,9 +106,11 @@ struct DraftSmemT : DraftSmem {};
 template <>
 struct DraftSmemT<true> : DraftSmem {
     float2 tab[kTabEntries];
+    double freq[64];  // w of every dimension pair
 };
 
-// kRope: q is rotated (RoPE) before its block mean.
+// kRope: q is rotated (RoPE) before its block mean (and, when a.q_rot is set,
+// the rotated q is stored there).
 template <bool kRope>
 __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
     __shared__ DraftSmemT<kRope> sm;
@@ -140,6 +143,8 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
         if constexpr (kRope) {
             // the block's rotation table, built while the loads above are in flight
+            if (tid < 64) sm.freq[tid] = rope_freq(tid, a.rope_base);
+            __syncthreads();
             for (int e = tid; e < kTabEntries; e += kThreads) {
                 int pos, pair;
                 if (e < kTabY) {
@@ -152,13 +157,14 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
                     pos = qbx * 8 + (e - kTabX) / kRopePairsY;
                     pair = kRopeFirstX + (e - kTabX) % kRopePairsY;
                 }
-                sm.tab[e] = rope_cs(pos, rope_freq(pair, a.rope_base));
+                sm.tab[e] = rope_cs(pos, sm.freq[pair]);
             }
             __syncthreads();
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int n = warp * 16 + 2 * i + half;  // token (t, y, x) = (n / 64, n / 8 % 8, n % 8)
                 const uint32_t w4[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+                uint32_t r4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int pair = 4 * d8 + e;
@@ -167,7 +173,13 @@ __global__ void __launch_bounds__(kThreads, 6) draft_kernel(const DraftArgs a) {
                                   : axis == 1 ? kTabY + ((n >> 3) & 7) * kRopePairsY + pair - kRopeFirstY
                                               : kTabX + (n & 7) * kRopePairsY + pair - kRopeFirstX;
                     const float2 cs = sm.tab[idx];
-                    add_bf16x2(acc[2 * e], acc[2 * e + 1], rope_rotate(w4[e], cs.x, cs.y));
+                    r4[e] = rope_rotate(w4[e], cs.x, cs.y);
+                    add_bf16x2(acc[2 * e], acc[2 * e + 1], r4[e]);
+                }
+                if (a.q_rot) {
+                    const size_t tok = ((frame + (n >> 6)) * a.tok_h + qby * 8 + ((n >> 3) & 7)) * a.tok_w + qbx * 8 +
+                                       (n & 7);
+                    reinterpret_cast<uint4 *>(a.q_rot + tok * kHeadDim)[d8] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
                 }
             }
         } else {

@@ -117,6 +117,7 @@ struct DraftArgs {
     int32_t *status;
     float rope_base;       // 0: no rotation of q
     int32_t rope_frame0;   // stream position of q's first frame
+    uint16_t *q_rot;       // may be null: receives the rotated q (with rope_base != 0)
 };
 
 cudaError_t launch_draft(const DraftArgs &a, bool pdl, const DeviceInfo &dev, cudaStream_t stream);

@@ -311,11 +311,20 @@ int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok
 }
 
 int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache *cache, int32_t *kept_idx,
-                    int32_t *kept_cnt, float *scores_opt, float *qmean_opt, int32_t *d_status, void *stream) {
+                    int32_t *kept_cnt, float *scores_opt, float *qmean_opt, void *q_rot_opt, int32_t *d_status,
+                    void *stream) {
     int rc = check_cache(cache);
     if (rc != LCSA_OK) return rc;
     if ((rc = check_params(p, cache)) != LCSA_OK) return rc;
     if (!q_tok || !aligned16(q_tok) || !kept_idx || !kept_cnt) return LCSA_ERR_INVALID_ARG;
+    if (q_rot_opt) {
+        // the rotated copy of q: only with a rotation, aligned, and apart from q
+        const size_t bytes = static_cast<size_t>(p->heads) * 2 * p->q_layers * 64 * p->grid_h * p->grid_w *
+                             LCSA_HEAD_DIM * 2;
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(q_tok), b0 = reinterpret_cast<uintptr_t>(q_rot_opt);
+        if (p->rope.base == 0.f || !aligned16(q_rot_opt) || (b0 < a0 + bytes && a0 < b0 + bytes))
+            return LCSA_ERR_INVALID_ARG;
+    }
     const int64_t cand = max_candidates(p, cache);
     if (cand > lcsa::kMaxCandidates) return LCSA_ERR_INVALID_ARG;
     const lcsa::DeviceInfo *dev = nullptr;
@@ -359,6 +368,7 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
     a.status = d_status;
     a.rope_base = p->rope.base;
     a.rope_frame0 = p->rope.frame0;
+    a.q_rot = static_cast<uint16_t *>(q_rot_opt);
     if (lcsa::launch_draft(a, (p->flags & LCSA_FLAG_PDL) != 0, *dev, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LCSA_ERR_CUDA;
     return LCSA_OK;

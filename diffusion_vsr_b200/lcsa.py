@@ -74,7 +74,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.lcsa_cache_append.argtypes = [P(lcsa_kv_cache), vp, vp, ctypes.c_int32, ctypes.c_int32, P(lcsa_rope), vp,
                                       vp]
     lib.lcsa_cache_append.restype = ctypes.c_int
-    lib.lcsa_draft_mask.argtypes = [P(lcsa_params), vp, P(lcsa_kv_cache), vp, vp, vp, vp, vp, vp]
+    lib.lcsa_draft_mask.argtypes = [P(lcsa_params), vp, P(lcsa_kv_cache), vp, vp, vp, vp, vp, vp, vp]
     lib.lcsa_draft_mask.restype = ctypes.c_int
     lib.lcsa_attention.argtypes = [P(lcsa_params), vp, P(lcsa_kv_cache), vp, vp, vp, vp, vp, vp]
     lib.lcsa_attention.restype = ctypes.c_int
@@ -171,9 +171,9 @@ def lcsa_cache_append(cache: KVCache, k_tok: torch.Tensor, v_tok: torch.Tensor, 
 def lcsa_draft_mask(params: lcsa_params, q_tok: torch.Tensor, cache: KVCache, kept_idx: torch.Tensor,
                     kept_cnt: torch.Tensor, scores: Optional[torch.Tensor] = None,
                     qmean: Optional[torch.Tensor] = None, d_status: Optional[torch.Tensor] = None,
-                    stream=None) -> None:
+                    stream=None, q_rot: Optional[torch.Tensor] = None) -> None:
     rc = load_library().lcsa_draft_mask(ctypes.byref(params), _ptr(q_tok), ctypes.byref(cache.desc),
-                                        _ptr(kept_idx), _ptr(kept_cnt), _ptr(scores), _ptr(qmean),
+                                        _ptr(kept_idx), _ptr(kept_cnt), _ptr(scores), _ptr(qmean), _ptr(q_rot),
                                         _ptr(d_status), _stream(stream))
     _check("lcsa_draft_mask", rc)
 
@@ -246,6 +246,11 @@ class LcsaLayer:
         # which writes q or the output, so both may launch as programmatic dependents
         self.params_chained = make_params(heads, grid_h, grid_w, q_layers, topk, local_range, local_mode,
                                           flags=LCSA_FLAG_PDL, rope_base=rope_base)
+        # with RoPE the draft stores the q it rotates, and the attention reads that
+        # copy without rotating again (params without a rotation)
+        self.params_attn = make_params(heads, grid_h, grid_w, q_layers, topk, local_range, local_mode,
+                                       flags=LCSA_FLAG_PDL)
+        self.q_rot: Optional[torch.Tensor] = None
         # kv_len + q_layers resident layers plus q_layers spare slots: a step's append
         # never overwrites a layer the previous step reads (see step(overlap_previous))
         self.cache = KVCache.allocate(kv_len + 2 * q_layers, heads, grid_h, grid_w, device,
@@ -279,8 +284,17 @@ class LcsaLayer:
         self.frame += k_tok.shape[1]
         self.params.rope.frame0 = frame0
         self.params_chained.rope.frame0 = frame0
-        lcsa_draft_mask(self.params_chained, q_tok, self.cache, self.kept_idx, self.kept_cnt, d_status=self.status)
-        lcsa_attention(self.params_chained, q_tok, self.cache, self.kept_idx, self.kept_cnt, out_tok, lse,
+        if not self.rope_base:
+            lcsa_draft_mask(self.params_chained, q_tok, self.cache, self.kept_idx, self.kept_cnt,
+                            d_status=self.status)
+            lcsa_attention(self.params_chained, q_tok, self.cache, self.kept_idx, self.kept_cnt, out_tok, lse,
+                           d_status=self.status)
+            return
+        if self.q_rot is None or self.q_rot.shape != q_tok.shape:
+            self.q_rot = torch.empty_like(q_tok)
+        lcsa_draft_mask(self.params_chained, q_tok, self.cache, self.kept_idx, self.kept_cnt, d_status=self.status,
+                        q_rot=self.q_rot)
+        lcsa_attention(self.params_attn, self.q_rot, self.cache, self.kept_idx, self.kept_cnt, out_tok, lse,
                        d_status=self.status)
 
 

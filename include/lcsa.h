@@ -61,7 +61,8 @@ enum lcsa_status {
                                      kernel that precedes the call in the stream,
                                      so that it starts while that kernel finishes.
                                      lcsa_draft_mask reads q_tok, writes
-                                     scores_opt / qmean_opt and reads the key
+                                     scores_opt / qmean_opt / q_rot_opt and
+                                     reads the key
                                      means of the layers older than the newest
                                      max(q_layers, cache->appended) before
                                      waiting for that kernel
@@ -71,7 +72,8 @@ enum lcsa_status {
                                      nothing before the wait.  Set the flag only
                                      when the preceding kernel neither writes
                                      q_tok or those older key means nor touches
-                                     scores_opt / qmean_opt, e.g. when it is the
+                                     scores_opt / qmean_opt / q_rot_opt, e.g.
+                                     when it is the
                                      cache append of the same chunk (before the
                                      draft: it writes only the cache->appended
                                      newest layers) or the draft (before the
@@ -189,11 +191,16 @@ int lcsa_cache_append(lcsa_kv_cache *cache, const void *k_tok, const void *v_tok
  *   scores_opt fp32 [heads][Nq][count*grid_h*grid_w] or NULL: s for allowed
  *              pairs, -inf elsewhere
  *   qmean_opt  fp32 [heads][Nq][128] or NULL: the q block means
+ *   q_rot_opt  bf16, q_tok's layout, or NULL; only with p->rope (else
+ *              LCSA_ERR_INVALID_ARG): receives q rotated (the values the
+ *              block means sum), so that lcsa_attention can read it with
+ *              rope.base = 0 instead of rotating q again.  16-byte aligned, not
+ *              overlapping q_tok.
  * Allowed candidates per row must not exceed LCSA_MAX_CANDIDATES.
  */
 int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache *cache,
                     int32_t *kept_idx, int32_t *kept_cnt, float *scores_opt,
-                    float *qmean_opt, int32_t *d_status, void *stream);
+                    float *qmean_opt, void *q_rot_opt, int32_t *d_status, void *stream);
 
 /*
  * lcsa_attention - block_sparse_attn_func of learn.html 2.2 (reading notes

@@ -100,6 +100,36 @@ def test_rope_1536x2688_sampled_rows_and_chained_launches():
         assert torch.equal(k1, k2) and torch.equal(o1, o2)
 
 
+def test_draft_stores_the_rotated_q_the_attention_reads():
+    # the draft's rotated copy of q is the oracle's rotation in the kernels'
+    # precision bit for bit, and the attention over it (without a rotation of its
+    # own) equals the attention that rotates the Q tiles itself, bit for bit
+    from diffusion_vsr_b200 import lcsa as L
+    from oracle import lcsa_oracle as O
+    w = W.WORKLOADS["768x1280"]
+    dev = torch.device("cuda")
+    layer = L.LcsaLayer(w.heads, w.grid_h, w.grid_w, w.q_layers, w.kv_len, w.topk, device=dev, rope_base=BASE)
+    for p in range(w.kv_len):
+        _, k, v = W.gen_layers(w, p, 1, "kv")
+        layer.append(k.to(dev), v.to(dev))
+    q, k, v = [t.to(dev) for t in W.gen_layers(w, w.kv_len, w.q_layers)]
+    frame0 = layer.frame
+    L.lcsa_cache_append(layer.cache, k, v, d_status=layer.status, rope=L.lcsa_rope(BASE, frame0))
+    layer.params.rope.frame0 = frame0
+    q_rot = torch.empty_like(q)
+    L.lcsa_draft_mask(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, d_status=layer.status,
+                      q_rot=q_rot)
+    out_self, out_read = torch.empty_like(q), torch.empty_like(q)
+    L.lcsa_attention(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, out_self, d_status=layer.status)
+    plain = L.make_params(w.heads, w.grid_h, w.grid_w, w.q_layers, w.topk)
+    L.lcsa_attention(plain, q_rot, layer.cache, layer.kept_idx, layer.kept_cnt, out_read, d_status=layer.status)
+    torch.cuda.synchronize()
+    assert layer.status.item() == 0
+    expected = O.apply_rope(q.float().cpu().numpy(), frame0, BASE, "kernel")
+    assert np.array_equal(q_rot.float().cpu().numpy(), expected)
+    assert torch.equal(out_self, out_read)
+
+
 def test_rope_changes_the_result():
     # positive control: the rotation is applied (outputs differ from the unrotated path)
     w = W.WORKLOADS["tiny"]

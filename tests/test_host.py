@@ -71,7 +71,7 @@ def test_cache_appended_field_is_validated(lib):
     p = L.make_params(2, 4, 4, 1, 8)
     for bad in (-1, 5):
         c = _fake_cache(appended=bad)
-        assert lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None) == \
+        assert lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None, None) == \
             L.LCSA_ERR_INVALID_ARG
         assert lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 1, 0, None, None, None) == \
             L.LCSA_ERR_INVALID_ARG
@@ -116,7 +116,7 @@ def test_draft_and_attention_reject_bad_params(lib, field, value):
     setattr(p, field, value)
     c = _fake_cache()
     z = ctypes.c_void_p(0x60000)
-    assert lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None) == \
+    assert lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None, None) == \
         L.LCSA_ERR_INVALID_ARG
     assert lib.lcsa_attention(ctypes.byref(p), z, ctypes.byref(c), z, z, ctypes.c_void_p(0x70000), None, None,
                               None) == L.LCSA_ERR_INVALID_ARG
@@ -130,7 +130,7 @@ def test_rope_arguments_are_validated(lib):
                              (float("inf"), 0, False), (10000.0, -1, False), (10000.0, (1 << 20) - 2, True),
                              (10000.0, (1 << 20) - 1, False)]:
         p = L.make_params(2, 4, 4, 1, 8, rope_base=base, rope_frame0=frame0)
-        rc = lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None)
+        rc = lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None, None)
         assert (rc != L.LCSA_ERR_INVALID_ARG) == ok, (base, frame0, rc)
         r = L.lcsa_rope(base, frame0)
         rc = lib.lcsa_cache_append(ctypes.byref(c), 0x40000, 0x50000, 1, 0, ctypes.byref(r), None, None)
@@ -138,12 +138,28 @@ def test_rope_arguments_are_validated(lib):
             assert rc == L.LCSA_ERR_INVALID_ARG, (base, frame0)
 
 
+@no_gpu_only
+def test_draft_rotated_q_needs_a_rotation_alignment_and_its_own_memory(lib):
+    q = 0x4000000  # 2 heads x 2 frames x 32 x 32 tokens x 128 dims bf16 = 1 MiB
+    z = ctypes.c_void_p(0x60000)
+    c = _fake_cache()
+    call = lambda p, q_rot: lib.lcsa_draft_mask(ctypes.byref(p), ctypes.c_void_p(q), ctypes.byref(c), z, z, None,
+                                                None, ctypes.c_void_p(q_rot), None, None)
+    assert call(L.make_params(2, 4, 4, 1, 8), 0x1000000) == L.LCSA_ERR_INVALID_ARG  # no rotation
+    p = L.make_params(2, 4, 4, 1, 8, rope_base=10000.0)
+    assert call(p, 0x1000008) == L.LCSA_ERR_INVALID_ARG  # misaligned
+    assert call(p, q + (1 << 20) - 16) == L.LCSA_ERR_INVALID_ARG  # overlaps q's last 16 bytes
+    assert call(p, q - (1 << 20) + 16) == L.LCSA_ERR_INVALID_ARG  # overlaps q's first 16 bytes
+    assert call(p, q + (1 << 20)) != L.LCSA_ERR_INVALID_ARG  # right after q: accepted
+    assert call(p, q - (1 << 20)) != L.LCSA_ERR_INVALID_ARG  # right before q: accepted
+
+
 def test_draft_rejects_too_many_candidates(lib):
     # no window over a 64 x 64 block grid: 4096 per layer x 4 layers > 4096
     p = L.make_params(1, 64, 64, 1, 8, local_range=0)
     c = _fake_cache(heads=1, grid_h=64, grid_w=64)
     z = ctypes.c_void_p(0x60000)
-    assert lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None) == \
+    assert lib.lcsa_draft_mask(ctypes.byref(p), z, ctypes.byref(c), z, z, None, None, None, None, None) == \
         L.LCSA_ERR_INVALID_ARG
 
 
