@@ -237,7 +237,7 @@ bool make_ring_map(CUtensorMap *m, const void *base, int64_t rows) {
 
 extern "C" {
 
-int lcsa_version(void) { return 101; }
+int lcsa_version(void) { return 102; }
 
 const char *lcsa_status_string(int code) {
     switch (code) {

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.lcsa_version() == 101
+    assert lib.lcsa_version() == 102
     assert L.status_string(L.LCSA_OK) == "LCSA_OK"
     assert L.status_string(L.LCSA_ERR_TIMEOUT) == "LCSA_ERR_TIMEOUT"
     assert L.status_string(L.LCSA_ERR_BAD_INDEX | L.LCSA_ERR_TIMEOUT).startswith("LCSA_ERR_TIMEOUT|")
