@@ -118,6 +118,9 @@ struct DraftArgs {
     float rope_base;       // 0: no rotation of q
     int32_t rope_frame0;   // stream position of q's first frame
     uint16_t *q_rot;       // may be null: receives the rotated q (with rope_base != 0)
+    // groups of query blocks (one CTA each): tile_h x tile_w blocks of one head
+    // and query layer, tiles_y x tiles_x groups per layer (set by launch_draft)
+    int32_t tile_h, tile_w, tiles_y, tiles_x;
 };
 
 cudaError_t launch_draft(const DraftArgs &a, bool pdl, const DeviceInfo &dev, cudaStream_t stream);
