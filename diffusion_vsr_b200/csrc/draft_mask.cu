@@ -31,13 +31,14 @@
 //     chained after the chunk's cache append, the keys of the older layers
 //     are scored while the append still runs, those of the chunk's own layers
 //     after it;
-//  3. exact top-k of every block of the group: scores become 32-bit keys
+//  3. exact top-k of every block of the group (two blocks: one half of the
+//     CTA each, at the same time): scores become 32-bit keys
 //     whose unsigned order is the descending score order; a radix select of
 //     up to 4 passes (8 bits per pass, block histogram in shared memory, one
 //     atomic per distinct bin and warp; it stops after the pass whose bin
-//     holding the k-th key is kept whole) finds the k-th key T; warp 0 writes
-//     every key < T plus the first (lowest-index) keys equal to T, in
-//     ascending key index, by a ballot compaction.
+//     holding the k-th key is kept whole) finds the k-th key T; the team's
+//     first warp writes every key < T plus the first (lowest-index) keys
+//     equal to T, in ascending key index, by a ballot compaction.
 
 #include <cfloat>
 #include <climits>
@@ -114,8 +115,8 @@ template <bool kRope, int kR>
 struct DraftSmem : RopeSmem<kRope> {
     __align__(16) float part[kWarps][kHeadDim];  // per-warp partial sums of q
     __align__(16) float mq[kR][kHeadDim];
-    uint32_t hist[256];
-    uint32_t digit, below, whole;
+    uint32_t hist[kR][256];  // radix histogram of each select team
+    uint32_t digit[kR], below[kR], whole[kR];
 };
 
 // Dot products of 8 keys with the group's kR q means, summed over the 32 lanes
@@ -373,10 +374,20 @@ __global__ void __launch_bounds__(kThreads, kR == 1 ? 6 : 4) draft_kernel(const 
     score_range(u_split, nu);
 
     // ---- 3. exact top-k of every block of the group: radix select of the k-th
-    //         smallest key, then the kept list in ascending key index
+    //         smallest key, then the kept list in ascending key index.  With two
+    //         blocks each half of the CTA (a team of 4 warps, its own histogram
+    //         and named barrier) selects one of them, the two at the same time.
+    __syncthreads();  // every block's candidates are complete
+    const int team_warps = kWarps / nb;
+    const int team = warp / team_warps;  // = the block this team selects
+    const int twarp = warp - team * team_warps;
+    const int tthreads = team_warps * 32;
+    const int ttid = tid - team * tthreads;
+    const uint32_t bar_id = 1u + static_cast<uint32_t>(team);
     const uint32_t lt_mask = lanemask_lt();
-#pragma unroll 1
-    for (int b = 0; b < nb; ++b) {
+    uint32_t *hist = sm.hist[team];
+    {
+        const int b = team;
         int x0, x1;
         window_1d(qbx0 + b, a.grid_w, a.local_range, a.local_mode, x0, x1);
         const int wx = x1 - x0;
@@ -389,23 +400,23 @@ __global__ void __launch_bounds__(kThreads, kR == 1 ? 6 : 4) draft_kernel(const 
 #pragma unroll 1
         for (int pass = 0; pass < 4; ++pass) {
             const int shift = 24 - 8 * pass;
-            sm.hist[tid] = 0u;  // kThreads == 256 bins
-            __syncthreads();    // (first pass: also the keys of phase 2)
-            for (int c0 = warp * 32; c0 < ncand; c0 += kThreads) {  // whole warps, one add per distinct bin
+            for (int i = ttid; i < 256; i += tthreads) hist[i] = 0u;
+            named_bar_sync(bar_id, tthreads);
+            for (int c0 = twarp * 32; c0 < ncand; c0 += tthreads) {  // whole warps, one add per distinct bin
                 const int c = c0 + lane;
                 const uint32_t key = c < ncand ? bk[c] : 0u;
                 const bool hit = c < ncand && (key & mask) == prefix;
                 const uint32_t bin = hit ? ((key >> shift) & 255u) : 256u;
                 const uint32_t peers = __match_any_sync(kFull, bin);
-                if (hit && (peers & lt_mask) == 0u) atomicAdd(&sm.hist[bin], static_cast<uint32_t>(__popc(peers)));
+                if (hit && (peers & lt_mask) == 0u) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
             }
-            __syncthreads();
-            if (warp == 0) {
+            named_bar_sync(bar_id, tthreads);
+            if (twarp == 0) {
                 uint32_t cnt[8];
                 uint32_t sum = 0;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    cnt[e] = sm.hist[lane * 8 + e];
+                    cnt[e] = hist[lane * 8 + e];
                     sum += cnt[e];
                 }
                 uint32_t incl = sum;
@@ -420,26 +431,26 @@ __global__ void __launch_bounds__(kThreads, kR == 1 ? 6 : 4) draft_kernel(const 
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         if (run + cnt[e] >= k_rem) {
-                            sm.digit = static_cast<uint32_t>(lane * 8 + e);
-                            sm.below = run;
-                            sm.whole = run + cnt[e] == k_rem;  // every key of the bin is kept
+                            sm.digit[team] = static_cast<uint32_t>(lane * 8 + e);
+                            sm.below[team] = run;
+                            sm.whole[team] = run + cnt[e] == k_rem;  // every key of the bin is kept
                             break;
                         }
                         run += cnt[e];
                     }
                 }
             }
-            __syncthreads();
-            k_rem -= sm.below;
-            prefix |= sm.digit << shift;
+            named_bar_sync(bar_id, tthreads);
+            k_rem -= sm.below[team];
+            prefix |= sm.digit[team] << shift;
             mask |= 255u << shift;
-            if (sm.whole) {  // the k-th key's bin is kept whole: no further digit is needed
+            if (sm.whole[team]) {  // the k-th key's bin is kept whole: no further digit is needed
                 prefix |= (1u << shift) - 1u;  // T = the largest key of the bin
                 whole = true;
                 break;
             }
         }
-        if (warp != 0) continue;  // (the next block's first barrier waits for warp 0)
+        if (twarp != 0) return;
         const uint32_t T = prefix;
         // keys equal to T that belong to the k smallest (all of them when the bin is kept whole)
         const int k_eq = whole ? INT_MAX : static_cast<int>(k_rem);
