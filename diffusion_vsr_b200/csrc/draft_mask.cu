@@ -383,7 +383,15 @@ __global__ void __launch_bounds__(kThreads, kR == 1 ? 6 : 4) draft_kernel(const 
     const int twarp = warp - team * team_warps;
     const int tthreads = team_warps * 32;
     const int ttid = tid - team * tthreads;
-    const uint32_t bar_id = 1u + static_cast<uint32_t>(team);
+    auto team_sync = [&]() {
+        if constexpr (kR == 1) {
+            __syncthreads();
+        } else if (team == 0) {
+            bar_sync_id<1>(tthreads);
+        } else {
+            bar_sync_id<2>(tthreads);
+        }
+    };
     const uint32_t lt_mask = lanemask_lt();
     uint32_t *hist = sm.hist[team];
     {
@@ -401,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, kR == 1 ? 6 : 4) draft_kernel(const 
         for (int pass = 0; pass < 4; ++pass) {
             const int shift = 24 - 8 * pass;
             for (int i = ttid; i < 256; i += tthreads) hist[i] = 0u;
-            named_bar_sync(bar_id, tthreads);
+            team_sync();
             for (int c0 = twarp * 32; c0 < ncand; c0 += tthreads) {  // whole warps, one add per distinct bin
                 const int c = c0 + lane;
                 const uint32_t key = c < ncand ? bk[c] : 0u;
@@ -410,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, kR == 1 ? 6 : 4) draft_kernel(const 
                 const uint32_t peers = __match_any_sync(kFull, bin);
                 if (hit && (peers & lt_mask) == 0u) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
             }
-            named_bar_sync(bar_id, tthreads);
+            team_sync();
             if (twarp == 0) {
                 uint32_t cnt[8];
                 uint32_t sum = 0;
@@ -440,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, kR == 1 ? 6 : 4) draft_kernel(const 
                     }
                 }
             }
-            named_bar_sync(bar_id, tthreads);
+            team_sync();
             k_rem -= sm.below[team];
             prefix |= sm.digit[team] << shift;
             mask |= 255u << shift;

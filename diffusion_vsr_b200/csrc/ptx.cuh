@@ -264,6 +264,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t m, uint32_t n, ui
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+// The same with the barrier as an immediate: ptxas then reserves only the
+// barriers a kernel names, not all 16 (which limits the CTAs per SM).
+template <int kId>
+__device__ __forceinline__ void bar_sync_id(uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"n"(kId), "r"(nthreads) : "memory");
+}
 
 // Per-warpgroup register budget changes (all warps of the warpgroup execute them).
 template <uint32_t N>
