@@ -179,10 +179,10 @@ __global__ void __launch_bounds__(kThreads, kR == 1 ? 6 : 4) draft_kernel(const 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     int t = blockIdx.x;  // (head, query layer, block row, group)
-    const int hq = t / (a.grid_h * a.tiles_x);
-    t -= hq * a.grid_h * a.tiles_x;
-    const int qby = t / a.tiles_x;
-    const int qbx0 = (t - qby * a.tiles_x) * kR;
+    const int hq = t / (a.grid_h * a.groups_x);
+    t -= hq * a.grid_h * a.groups_x;
+    const int qby = t / a.groups_x;
+    const int qbx0 = (t - qby * a.groups_x) * kR;
     const int nb = min(kR, a.grid_w - qbx0);  // blocks of the group: qbx0 .. qbx0 + nb - 1
     const int h = hq / a.q_layers, ql = hq - h * a.q_layers;
     const int unit0 = hq * a.nblk + qby * a.grid_w + qbx0;  // row of block b: unit0 + b
@@ -500,7 +500,7 @@ cudaError_t launch_group(const DraftArgs &a, bool pdl, const DeviceInfo &dev, cu
         const cudaError_t e = ensure_smem_limit(draft_kernel<kRope, kR>, dev.device, smem, smem_set);
         if (e != cudaSuccess) return e;
     }
-    const int grid = a.heads * a.q_layers * a.grid_h * a.tiles_x;
+    const int grid = a.heads * a.q_layers * a.grid_h * a.groups_x;
     return launch_kernel(draft_kernel<kRope, kR>, dim3(grid), dim3(kThreads), smem, stream, pdl, a);
 }
 
@@ -515,12 +515,10 @@ cudaError_t launch_draft(const DraftArgs &in, bool pdl, const DeviceInfo &dev, c
     constexpr int kGroupMinRows = 2048;
     DraftArgs a = in;
     const int64_t rows = static_cast<int64_t>(a.heads) * a.q_layers * a.nblk;
-    a.tile_h = 1;
-    a.tile_w = (a.grid_w >= 2 && rows >= kGroupMinRows) ? 2 : 1;
-    a.tiles_y = a.grid_h;
-    a.tiles_x = (a.grid_w + a.tile_w - 1) / a.tile_w;
+    const int group = (a.grid_w >= 2 && rows >= kGroupMinRows) ? 2 : 1;
+    a.groups_x = (a.grid_w + group - 1) / group;
     const bool rope = a.rope_base != 0.f;
-    if (a.tile_w == 2)
+    if (group == 2)
         return rope ? launch_group<true, 2>(a, pdl, dev, stream) : launch_group<false, 2>(a, pdl, dev, stream);
     return rope ? launch_group<true, 1>(a, pdl, dev, stream) : launch_group<false, 1>(a, pdl, dev, stream);
 }

@@ -108,7 +108,6 @@ struct DraftArgs {
     int32_t fresh_layers;  // newest layers the preceding kernel may still be writing (PDL)
     int32_t local_range, local_mode, topk;
     int32_t cand_cap;      // most allowed candidates of a row, rounded up to 32
-    uint64_t m_nq, m_nblk, m_gw;  // multiply-high multipliers of q_layers*nblk, nblk, grid_w
     float scale;
     int32_t *kept_idx;
     int32_t *kept_cnt;
@@ -118,9 +117,9 @@ struct DraftArgs {
     float rope_base;       // 0: no rotation of q
     int32_t rope_frame0;   // stream position of q's first frame
     uint16_t *q_rot;       // may be null: receives the rotated q (with rope_base != 0)
-    // groups of query blocks (one CTA each): tile_h x tile_w blocks of one head
-    // and query layer, tiles_y x tiles_x groups per layer (set by launch_draft)
-    int32_t tile_h, tile_w, tiles_y, tiles_x;
+    // groups of horizontally adjacent query blocks (one CTA each) per block
+    // row of a layer (set by launch_draft)
+    int32_t groups_x;
 };
 
 cudaError_t launch_draft(const DraftArgs &a, bool pdl, const DeviceInfo &dev, cudaStream_t stream);

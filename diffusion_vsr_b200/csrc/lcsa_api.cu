@@ -351,15 +351,6 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
     a.local_mode = p->local_mode;
     a.topk = p->topk;
     a.cand_cap = static_cast<int32_t>((cand + 31) / 32 * 32);
-    {
-        // row decomposition by multiply-high division, exact while dividend x divisor <= 2^32
-        const int64_t nq = static_cast<int64_t>(p->q_layers) * a.nblk;
-        if (static_cast<int64_t>(p->heads) * nq * nq > (1ll << 32) || nq * a.nblk > (1ll << 32))
-            return LCSA_ERR_INVALID_ARG;
-        a.m_nq = lcsa::div_magic_host(static_cast<uint32_t>(nq));
-        a.m_nblk = lcsa::div_magic_host(static_cast<uint32_t>(a.nblk));
-        a.m_gw = lcsa::div_magic_host(static_cast<uint32_t>(a.grid_w));
-    }
     a.scale = eff_scale(p);
     a.kept_idx = kept_idx;
     a.kept_cnt = kept_cnt;
