@@ -259,6 +259,11 @@ def measure_lcsa(w: W.Workload, args, world: int, local_rank: int, dev, with_e2e
         layer.append(k.to(dev), v.to(dev))
     out = torch.empty_like(chunks[0][0])
     stream = torch.cuda.current_stream(dev)
+    # with RoPE, the attention of the per-kernel pass reads the draft's rotated q
+    # without a rotation of its own, as LcsaLayer.step does
+    plain_params = L.make_params(w.heads, w.grid_h, w.grid_w, w.q_layers, w.topk, w.local_range, w.local_mode)
+    if args.rope:
+        layer.q_rot = torch.empty_like(chunks[0][0])
 
     def step(i):
         # the library's streaming step, chained: the append runs in the SMs the
@@ -278,13 +283,9 @@ def measure_lcsa(w: W.Workload, args, world: int, local_rank: int, dev, with_e2e
         layer.frame += k.shape[1]
         ev[1].record(stream)
         if args.rope:
-            # as LcsaLayer.step: the draft stores the rotated q, the attention reads it
-            if layer.q_rot is None:
-                layer.q_rot = torch.empty_like(q)
             L.lcsa_draft_mask(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, d_status=layer.status,
                               q_rot=layer.q_rot)
-            attn_params, attn_q = L.make_params(w.heads, w.grid_h, w.grid_w, w.q_layers, w.topk, w.local_range,
-                                                w.local_mode), layer.q_rot
+            attn_params, attn_q = plain_params, layer.q_rot
         else:
             L.lcsa_draft_mask(layer.params, q, layer.cache, layer.kept_idx, layer.kept_cnt, d_status=layer.status)
             attn_params, attn_q = layer.params, q

@@ -255,6 +255,22 @@ def test_bench_main_exits_nonzero_on_world_mismatch():
     assert r.returncode != 0 and "WORLD_SIZE=1" in r.stderr
 
 
+def test_bench_rope_and_segment_options():
+    import bench
+    from diffusion_vsr_b200 import workloads as W
+    a = bench.parse_args(["--rope", "10000", "--segments", "768x1280"])
+    assert a.rope == 10000.0 and a.segments == "768x1280"
+    assert bench.parse_args([]).rope == 0.0 and bench.parse_args([]).segments is None
+    w = W.WORKLOADS["768x1408"]
+    # the default line's config carries no RoPE key, so both arms print the same dict
+    assert "rope_base" not in bench.bench_config(w, 15840, 1)
+    assert bench.bench_config(w, 15840, 1, rope=10000.0)["rope_base"] == 10000.0
+    # the segment line's work: every (query tile, key tile) pair of a segment
+    sw = W.SEGMENT_WORKLOADS[bench.SWEEP_SEGMENTS]
+    assert sw.seg_tiles == [30, 150, 30, 90]
+    assert sw.kept_tiles == 12 * (30 ** 2 + 150 ** 2 + 30 ** 2 + 90 ** 2) == 388800
+
+
 def test_bench_config_is_shared_by_both_arms():
     import bench
     from diffusion_vsr_b200 import workloads as W
