@@ -215,7 +215,10 @@ int lcsa_draft_mask(const lcsa_params *p, const void *q_tok, const lcsa_kv_cache
  *   lse_opt  fp32 [heads][2*q_layers][8*grid_h][8*grid_w] or NULL: natural
  *            log of the softmax denominator of each query token
  * With p->rope, the Q tiles are rotated (lcsa_rope) before the products (the
- * keys were rotated by the cache append).
+ * keys were rotated by the cache append).  That rotation runs inside the
+ * kernel on every Q tile; the faster path, when lcsa_draft_mask runs first,
+ * is its q_rot_opt copy passed here as q_tok with rope.base = 0: the same
+ * rotated values, bit for bit, and no rotation left in this kernel.
  * A row with kept_cnt == 0 gets zeros (lse -inf).  A kept index outside
  * [0, count*grid_h*grid_w) or a count outside [0, topk] sets
  * LCSA_ERR_BAD_INDEX and the row is written as if it kept nothing.
